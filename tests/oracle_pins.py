@@ -1,0 +1,436 @@
+"""Pins that tie the CPU oracle to facts outside itself.
+
+Each pin takes the oracle module as an argument (so the mutation test can run
+the same pins against a copy of the oracle with a planted mistake) and raises
+AssertionError when the oracle disagrees with:
+  * values the source pages print (tests/golden/*.txt, each with its citation),
+  * a hand-worked example (tests/golden/hand_worked_scores.json),
+  * brute force on tiny inputs (Python integers, subset enumeration),
+  * closed forms and invariants of the definitions,
+  * library routines for the storage formats (torch's float8/bfloat16 casts,
+    Python sets, exact rationals).
+"""
+
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rows(name):
+    out = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                out.append([int(x) for x in line.split()])
+    return out
+
+
+def _bf16_bits_of_ints(a) -> np.ndarray:
+    """Small integers -> bf16 bit patterns via torch (exact for |x| <= 256)."""
+    t = torch.tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _problem(S, T, H, D, K, vis=0, ratio=1, dtype="bf16", q_pos0=0):
+    return dict(S=S, T=T, H=H, D=D, K=K, visibility=vis, ratio=ratio,
+                dtype=dtype, q_pos0=q_pos0)
+
+
+def _beats(a, b):
+    """(score, index) a is ranked above b: higher score, then lower index."""
+    return a[0] > b[0] or (a[0] == b[0] and a[1] < b[1])
+
+
+# ----------------------------------------------------------------------------
+# score arithmetic
+# ----------------------------------------------------------------------------
+
+def pin_hand_worked(O):
+    with open(os.path.join(GOLDEN, "hand_worked_scores.json")) as f:
+        ex = json.load(f)
+    q = np.array(ex["q"], dtype=np.float64)
+    w = np.array(ex["w"], dtype=np.float64)
+    keys = np.array(ex["keys"], dtype=np.float64)
+    s = O.score_keys(q, w, keys)
+    assert s.tolist() == [float(x) for x in ex["scores"]], s
+    qb = _bf16_bits_of_ints(q)[None]
+    kb = _bf16_bits_of_ints(keys)
+    for case in ex["cases"]:
+        g, K = case["g"], case["K"]
+        prob = _problem(S=g + 1, T=len(keys), H=ex["H"], D=ex["D"], K=K)
+        idx, ln, sc, tau = O.topk_rows(prob, qb, kb, w[None].astype(np.float32), [g])
+        assert int(ln[0]) == len(case["idx"]), (case, ln)
+        assert idx[0, : ln[0]].tolist() == case["idx"], (case, idx)
+        assert (idx[0, ln[0]:] == -1).all()
+
+
+def pin_integer_bruteforce(O):
+    rng = np.random.default_rng(7)
+    for trial in range(6):
+        H, D, n = int(rng.integers(1, 5)), int(rng.integers(1, 9)), 16
+        q = rng.integers(-3, 4, size=(H, D))
+        w = rng.integers(-2, 3, size=H)
+        keys = rng.integers(-3, 4, size=(n, D))
+        expect = []
+        for i in range(n):
+            tot = 0
+            for h in range(H):
+                dot = 0
+                for d in range(D):
+                    dot += int(q[h, d]) * int(keys[i, d])
+                tot += int(w[h]) * max(dot, 0)
+            expect.append(tot)
+        got = O.score_keys(q.astype(np.float64), w.astype(np.float64), keys.astype(np.float64))
+        assert got.tolist() == [float(x) for x in expect], (trial, got, expect)
+
+
+def pin_score_properties(O):
+    rng = np.random.default_rng(11)
+    H, D, n = 5, 16, 40
+    q = rng.standard_normal((H, D))
+    w = rng.standard_normal(H)
+    keys = rng.standard_normal((n, D))
+    s = O.score_keys(q, w, keys)
+    # positive homogeneity in the key and in the weights
+    assert np.allclose(O.score_keys(q, w, 2.0 * keys), 2.0 * s, rtol=1e-12, atol=1e-12)
+    assert np.allclose(O.score_keys(q, -w, keys), -s, rtol=1e-12, atol=1e-12)
+    # the score is linear in w: s(w1 + w2) = s(w1) + s(w2)
+    w2 = rng.standard_normal(H)
+    assert np.allclose(O.score_keys(q, w + w2, keys), s + O.score_keys(q, w2, keys), rtol=1e-10, atol=1e-10)
+    # heads are interchangeable when q rows and weights move together
+    perm = rng.permutation(H)
+    assert np.allclose(O.score_keys(q[perm], w[perm], keys), s, rtol=1e-12, atol=1e-12)
+    # one head with weight 1: s = max(0, q.k); a key opposite to q scores 0
+    e0 = np.zeros(H)
+    e0[0] = 1.0
+    s0 = O.score_keys(q, e0, keys)
+    assert np.allclose(s0, np.maximum(keys @ q[0], 0.0), rtol=1e-12, atol=1e-12)
+    assert O.score_keys(q, e0, -q[:1])[0] == 0.0
+    # a negative weight on an active head lowers the score
+    e1 = np.zeros(H)
+    e1[1] = -1.0
+    assert O.score_keys(q, e1, q[1:2])[0] < 0
+
+
+# ----------------------------------------------------------------------------
+# selection
+# ----------------------------------------------------------------------------
+
+def pin_selection_bruteforce(O):
+    rng = np.random.default_rng(3)
+    for trial in range(60):
+        n = int(rng.integers(1, 11))
+        K = int(rng.integers(1, 6))
+        s = rng.integers(-2, 3, size=n).astype(np.float64)  # many ties
+        if trial % 3 == 0:
+            s = -s * 0.0  # all zero, some -0.0
+        keys = np.arange(n, dtype=np.int64)
+        m = min(K, n)
+        winners = []
+        for sub in itertools.combinations(range(n), m):
+            rest = [i for i in range(n) if i not in sub]
+            if all(_beats((s[a], a), (s[b], b)) for a in sub for b in rest):
+                winners.append(sub)
+        assert len(winners) == 1, (s, K, winners)
+        sel, ssel, tau = O.select_topk(s + 0.0, keys, K)
+        assert sel.tolist() == list(winners[0]), (trial, s, K, sel, winners)
+        assert ssel.tolist() == [s[i] + 0.0 for i in winners[0]]
+
+
+def pin_selection_dominance(O):
+    rng = np.random.default_rng(5)
+    n, K = 400, 57
+    s = np.round(rng.standard_normal(n) * 4) / 2  # ties on a 0.5 grid
+    keys = np.arange(n, dtype=np.int64) * 3 + 1     # ascending, not 0..n-1
+    sel, ssel, tau = O.select_topk(s, keys, K)
+    assert sel.size == K and np.all(np.diff(sel) > 0)
+    chosen = set(sel.tolist())
+    pos = {int(k): i for i, k in enumerate(keys)}
+    ins = [(s[pos[k]], k) for k in chosen]
+    outs = [(s[i], int(keys[i])) for i in range(n) if int(keys[i]) not in chosen]
+    for a in ins:
+        for b in outs:
+            assert _beats(a, b), (a, b)
+    kth = sorted(ins, key=lambda x: (-x[0], x[1]))[-1]
+    assert tau == kth[0]
+
+
+def pin_chunked_equals_materialised(O):
+    """StreamIndex (arXiv 2605.02568, abstract): a chunked partition-merge top-K
+    must reproduce the materialised result.  The chunked side here is an
+    independent tuple sort: per chunk keep the best K, then merge."""
+    rng = np.random.default_rng(9)
+    for trial in range(8):
+        n = int(rng.integers(50, 600))
+        K = int(rng.integers(1, 80))
+        chunk = int(rng.integers(7, 130))
+        s = np.round(rng.standard_normal(n) * 3)  # integer scores: ties
+        keys = np.arange(n, dtype=np.int64)
+        kept = []
+        for c0 in range(0, n, chunk):
+            part = [(-s[i], i) for i in range(c0, min(n, c0 + chunk))]
+            kept.extend(sorted(part)[:K])
+            kept = sorted(kept)[:K]
+        expect = sorted(i for _, i in kept)
+        sel, _, _ = O.select_topk(s, keys, K)
+        assert sel.tolist() == expect, (trial, n, K, chunk)
+
+
+def pin_row_invariants(O):
+    rng = np.random.default_rng(21)
+    H, D, T, K = 3, 8, 300, 40
+    qb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, H, D)))
+    kb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, D)))
+    w = rng.integers(-2, 3, size=(T, H)).astype(np.float32)
+    rows = np.arange(0, T, 7)
+    for vis, ratio in ((0, 1), (1, 4), (2, 4)):
+        prob = _problem(S=T, T=T, H=H, D=D, K=K, vis=vis, ratio=ratio)
+        idx, ln, sc, tau = O.topk_rows(prob, qb[rows], kb, w[rows], rows,
+                                       pool_coef=_bf16_bits_of_ints(np.ones((ratio, D))))
+        width = O.out_width(K, vis, ratio)
+        assert idx.shape == (rows.size, width)
+        for r, t in enumerate(rows):
+            g = int(t)
+            row = idx[r, : ln[r]]
+            assert np.all(np.diff(row) > 0), (vis, t, row)
+            assert np.all(idx[r, ln[r]:] == -1)
+            if vis == 0:
+                assert ln[r] == min(K, g + 1)
+                assert row.size == 0 or row[-1] <= g
+            elif vis == 1:
+                nv = min((g + 1) // ratio, T)
+                assert ln[r] == min(K, nv)
+                assert np.all(ratio * row + ratio - 1 <= g)
+            else:
+                nc = (g + 1) // ratio
+                assert ln[r] == ratio * min(K // ratio, nc) + (g + 1) % ratio
+                assert np.all(row <= g)
+
+
+def pin_prefix_closed_form(O):
+    """Token rows whose whole prefix fits in the budget select exactly 0..g."""
+    rng = np.random.default_rng(4)
+    H, D, T, K = 2, 4, 64, 16
+    qb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, H, D)))
+    kb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, D)))
+    w = rng.integers(-2, 3, size=(T, H)).astype(np.float32)
+    rows = np.arange(K)
+    idx, ln, _, _ = O.topk_rows(_problem(T, T, H, D, K), qb[rows], kb, w[rows], rows)
+    for g in range(K):
+        assert idx[g, : ln[g]].tolist() == list(range(g + 1))
+
+
+# ----------------------------------------------------------------------------
+# visibility, pooling, slots
+# ----------------------------------------------------------------------------
+
+def pin_visibility_closed_forms(O):
+    T = 50
+    for g in range(0, 230):
+        assert O.visible_keys(g, T, O.TOKEN, 1).tolist() == list(range(min(g + 1, T)))
+        for m in (1, 2, 4, 7):
+            v = O.visible_keys(g, T, O.COMPRESSED, m)
+            assert v.tolist() == list(range(min((g + 1) // m, T))), (g, m)
+            lit = [p for p in range(T) if all(m * p + j <= g for j in range(m))]
+            assert O.visible_keys(g, T, O.POOLED, m).tolist() == lit, (g, m)
+
+
+def pin_watch_lengths(O):
+    for L, pools, tail in _rows("kpool_watch_lengths.txt"):
+        g = L - 1
+        assert O.visible_keys(g, 1000, O.POOLED, 4).size == pools, L
+        assert O.incomplete_tail(g, 4).size == tail, L
+        assert O.incomplete_tail(g, 4).tolist() == list(range(4 * pools, g + 1))
+        # through the full row path, with a budget larger than the history
+        D = 2
+        kb = _bf16_bits_of_ints(np.ones((16, D)))
+        qb = _bf16_bits_of_ints(np.ones((1, 1, D)))
+        prob = _problem(S=g + 1, T=16, H=1, D=D, K=8, vis=O.POOLED, ratio=4)
+        idx, ln, _, _ = O.topk_rows(prob, qb, kb, np.ones((1, 1), np.float32), [g],
+                                    pool_coef=_bf16_bits_of_ints(np.ones((4, D))))
+        assert int(ln[0]) == 4 * pools + tail
+        assert idx[0, : ln[0]].tolist() == list(range(L)), (L, idx)
+
+
+def pin_slot_count(O):
+    budget, width, pools, slots = _rows("kpool_slots.txt")[0]
+    assert O.out_width(budget, O.POOLED, width) == slots
+    assert budget // width == pools
+    # a row that fills every slot: >= 512 complete pools and a 3-token tail
+    D, T = 2, 4 * 600
+    g = 4 * 515 + 2
+    kb = _bf16_bits_of_ints(np.ones((T, D)))
+    qb = _bf16_bits_of_ints(np.ones((1, 1, D)))
+    prob = _problem(S=g + 1, T=T, H=1, D=D, K=budget, vis=O.POOLED, ratio=width)
+    idx, ln, _, _ = O.topk_rows(prob, qb, kb, np.ones((1, 1), np.float32), [g],
+                                pool_coef=_bf16_bits_of_ints(np.ones((width, D))))
+    assert idx.shape[1] == slots and int(ln[0]) == slots
+
+
+def pin_pooled_keys(O):
+    rng = np.random.default_rng(13)
+    T, D, m = 40, 6, 4
+    kb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, D)))
+    # one-hot coefficients pick one constituent exactly
+    for j in range(m):
+        c = np.zeros((m, D))
+        c[j] = 1.0
+        kp = O.pooled_keys(kb, _bf16_bits_of_ints(c), m)
+        assert (kp == kb[j::m][: T // m]).all(), j
+    # unit coefficients: integer sums, exact
+    ints = rng.integers(-3, 4, size=(T, D))
+    kp = O.pooled_keys(_bf16_bits_of_ints(ints), _bf16_bits_of_ints(np.ones((m, D))), m)
+    expect = ints.reshape(T // m, m, D).sum(axis=1)
+    assert (kp == _bf16_bits_of_ints(expect)).all()
+    # general values against exact rationals and a nearest-value search
+    kf = torch.randn(T, D, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    cf = (torch.rand(m, D, generator=torch.Generator().manual_seed(2)) * 0.5).to(torch.bfloat16)
+    kbits = kf.view(torch.int16).numpy().view(np.uint16)
+    cbits = cf.view(torch.int16).numpy().view(np.uint16)
+    kp = O.pooled_keys(kbits, cbits, m)
+    kv, cv = kf.float().numpy(), cf.float().numpy()
+    for p in range(T // m):
+        for d in range(D):
+            exact = sum(Fraction(float(kv[m * p + j, d])) * Fraction(float(cv[j, d])) for j in range(m))
+            assert int(kp[p, d]) == _nearest_bf16_bits(exact), (p, d)
+
+
+def _nearest_bf16_bits(v: Fraction) -> int:
+    """Nearest bfloat16 to an exact rational (ties to the even pattern), found
+    by bisection over the ordered positive bit patterns, decoded by torch."""
+    if v == 0:
+        return 0
+    sign = 0x8000 if v < 0 else 0
+    a = abs(v)
+    pats = torch.arange(0, 0x7F80, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float().numpy()
+    lo, hi = 0, len(pats) - 1
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if Fraction(float(pats[mid])) <= a:
+            lo = mid
+        else:
+            hi = mid
+    dl = a - Fraction(float(pats[lo]))
+    dh = Fraction(float(pats[hi])) - a
+    if dl < dh or (dl == dh and lo % 2 == 0):
+        return sign | lo
+    return sign | hi
+
+
+# ----------------------------------------------------------------------------
+# storage formats against library casts
+# ----------------------------------------------------------------------------
+
+def pin_e4m3_decoder(O):
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.decode_e4m3(codes)
+    both_nan = np.isnan(ref) & np.isnan(got)
+    assert np.all(both_nan | (ref == got)), np.nonzero(~(both_nan | (ref == got)))
+    assert np.nanmax(got) == 448.0
+
+
+def pin_bf16_codec(O):
+    rng = np.random.default_rng(17)
+    bits = rng.integers(0, 1 << 16, size=20000).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]  # finite patterns
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.decode_bf16(bits), ref)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(3.0),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),            # subnormal
+        np.array([3.3e38, -3.39e38, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 0.0, -0.0], np.float32),
+    ])
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = O.round_to_bf16_bits(x.astype(np.float64))
+    assert np.array_equal(got, ref), np.nonzero(got != ref)
+    # binary64 inputs carrying bits beyond binary32 (sticky bits matter)
+    for v in (1.0 + 2 ** -8 + 2 ** -40, 1.0 + 2 ** -8 - 2 ** -40, -(3.0 + 2 ** -7 + 2 ** -50), 12345.678901234):
+        assert int(O.round_to_bf16_bits(np.array([v]))[0]) == _nearest_bf16_bits(Fraction(v)), v
+
+
+# ----------------------------------------------------------------------------
+# adjacent-pair overlap
+# ----------------------------------------------------------------------------
+
+def pin_pair_overlap(O):
+    rng = np.random.default_rng(23)
+    S, W = 40, 30
+    idx = np.full((S, W), -1, dtype=np.int32)
+    ln = np.zeros(S, dtype=np.int32)
+    for r in range(S):
+        n = int(rng.integers(0, W + 1))
+        row = np.sort(rng.choice(60, size=n, replace=False))
+        idx[r, :n] = row
+        ln[r] = n
+    got = O.pair_shared_counts(idx, ln)
+    assert got.size == S // 2
+    for p in range(S // 2):
+        a = set(idx[2 * p, : ln[2 * p]].tolist())
+        b = set(idx[2 * p + 1, : ln[2 * p + 1]].tolist())
+        assert got[p] == len(a & b), p
+    # nested causal prefixes: the even row is contained in the odd row
+    idx2 = np.full((6, 8), -1, np.int32)
+    ln2 = np.array([1, 2, 3, 4, 5, 6], np.int32)
+    for r in range(6):
+        idx2[r, : r + 1] = np.arange(r + 1)
+    assert O.pair_shared_counts(idx2, ln2).tolist() == [1, 3, 5]
+
+
+def pin_fp8_scales(O):
+    """An FP8 value means code * row scale: doubling every key scale doubles
+    every score and leaves the selection unchanged; a per-(query, head) scale
+    acts on that head exactly like its weight."""
+    rng = np.random.default_rng(29)
+    H, D, T, K = 3, 8, 64, 9
+    codes_q = rng.integers(0, 0x7E, size=(1, H, D)).astype(np.uint8)  # finite codes
+    codes_k = rng.integers(0, 0x7E, size=(T, D)).astype(np.uint8)
+    codes_q[..., ::2] |= 0x80
+    codes_k[::3] |= 0x80
+    w = np.array([[0.5, -1.0, 2.0]], dtype=np.float32)
+    prob = _problem(S=1, T=T, H=H, D=D, K=K, dtype="fp8", q_pos0=T - 1)
+    one = np.ones(T, np.float32)
+    qs = np.ones((1, H), np.float32)
+    i1, l1, s1, _ = O.topk_rows(prob, codes_q, codes_k, w, [0], q_scale_rows=qs, k_scale=one)
+    i2, l2, s2, _ = O.topk_rows(prob, codes_q, codes_k, w, [0], q_scale_rows=qs, k_scale=2 * one)
+    assert np.array_equal(i1, i2) and np.allclose(s2[0, : l2[0]], 2 * s1[0, : l1[0]], rtol=1e-12)
+    qs2 = np.array([[2.0, 1.0, 1.0]], np.float32)
+    w2 = np.array([[0.25, -1.0, 2.0]], np.float32)
+    i3, l3, s3, _ = O.topk_rows(prob, codes_q, codes_k, w2, [0], q_scale_rows=qs2, k_scale=one)
+    assert np.array_equal(i1, i3) and np.allclose(s3[0, : l3[0]], s1[0, : l1[0]], rtol=1e-12)
+    # and the decoded value equals the library's cast times the scale
+    k64 = torch.from_numpy(codes_k.copy()).view(torch.float8_e4m3fn).double().numpy()
+    q64 = torch.from_numpy(codes_q.copy()).view(torch.float8_e4m3fn).double().numpy()[0]
+    s_lib = np.maximum(k64 @ q64.T, 0.0) @ w[0].astype(np.float64)
+    top = np.argsort(-s_lib, kind="stable")[:K]
+    assert i1[0, : l1[0]].tolist() == sorted(top.tolist())
+
+
+PINS = [
+    pin_hand_worked,
+    pin_integer_bruteforce,
+    pin_score_properties,
+    pin_selection_bruteforce,
+    pin_selection_dominance,
+    pin_chunked_equals_materialised,
+    pin_row_invariants,
+    pin_prefix_closed_form,
+    pin_visibility_closed_forms,
+    pin_watch_lengths,
+    pin_slot_count,
+    pin_pooled_keys,
+    pin_e4m3_decoder,
+    pin_bf16_codec,
+    pin_pair_overlap,
+    pin_fp8_scales,
+]
