@@ -1,0 +1,316 @@
+"""Benchmark of the indexer hot path (score + top-K + finalise) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one indexer_topk call over the whole workload (every query row),
+inputs resident in HBM.  Prints one JSON line (rank 0).  Under torchrun each
+rank runs its own independent problem of the same shape (weak scaling); the
+time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from head_weighted_relu_b200 import workloads as W  # noqa: E402
+
+METRIC = "indexer Gpairs/s (causal q·k pairs scored+top-K'd) & % tensor peak; peak HBM GB"
+L2_BYTES = 126 * 2 ** 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+                self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def flops_per_pair(wl):
+    return 2.0 * wl.H * wl.D
+
+
+def cpu_baseline(wl, seconds=15.0, max_rows=None):
+    """The oracle as it stands, timed on this host's cores on a bounded sample:
+    query rows at the end of the workload's query range (the rows that see the
+    most keys), drawn with the workload's shapes and distributions."""
+    import oracle
+    from head_weighted_relu_b200 import indexer as I
+    n = 64
+    sub = wl.scaled(S=n, q_pos0=wl.q_pos0 + wl.S - n)
+    inp = W.generate(sub, "cpu")
+    prob = sub.problem()
+    hk = W.to_host_bits(inp["k"])
+    ks = W.to_host_bits(inp["k_scale"])
+    pc = W.to_host_bits(inp["pool_coef"])
+    keys = oracle.decode_keys_for(prob, hk, ks, pc)
+    done, pairs, t0 = 0, 0, time.perf_counter()
+    for t in range(n - 1, -1, -1):
+        qs = None if inp["q_scale"] is None else W.to_host_bits(inp["q_scale"][t:t + 1])
+        oracle.topk_rows(prob, W.to_host_bits(inp["q"][t:t + 1]), hk, W.to_host_bits(inp["w"][t:t + 1]),
+                         np.array([t]), q_scale_rows=qs, k_scale=ks, pool_coef=pc, keys_f64=keys)
+        pairs += I.visible_pairs(1, sub.T, sub.visibility, sub.ratio, sub.q_pos0 + t)
+        done += 1
+        if time.perf_counter() - t0 > seconds or (max_rows and done >= max_rows):
+            break
+    dt = time.perf_counter() - t0
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count()
+    return dict(value=pairs / dt / 1e9, unit="Gpairs/s", cores=cores, kind="oracle",
+                sample=f"the last {done} query rows of {wl.name} ({pairs} pairs, {dt:.1f} s); "
+                       "NumPy FP64, full score row + stable sort per row, multithreaded BLAS")
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    base = cpu_baseline(wl, seconds=5.0)
+    steps = []
+    for _ in range(args.warmup):
+        cpu_baseline(wl, seconds=2.0, max_rows=2)
+    for _ in range(args.steps):
+        steps.append(cpu_baseline(wl, seconds=5.0))
+    val = statistics.median(s["value"] for s in steps)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "Gpairs/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "S": wl.S, "T": wl.T, "H": wl.H, "D": wl.D, "K": wl.K},
+        "cpu_baseline": dict(base, value=val),
+        "e2e": {"value": val, "unit": "Gpairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dsa_prefill_64k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    wl = W.WORKLOADS[args.workload]
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    from head_weighted_relu_b200 import indexer as I
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl_r = wl.scaled(seed=wl.seed + 1000 * rank)
+    inp = W.generate(wl_r, dev)
+    prob = I.make_problem(wl.S, wl.T, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype, wl.q_pos0)
+    bufs = I.allocate(prob, dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        I.topk(inp["q"], inp["k"], inp["w"], wl.K, visibility=wl.visibility, ratio=wl.ratio,
+               q_pos0=wl.q_pos0, q_scale=inp["q_scale"], k_scale=inp["k_scale"],
+               pool_coef=inp["pool_coef"], buffers=bufs, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = I.indexer_read_status(bufs[3])
+
+    # ---- timed region: K steps, events per step on the launching stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    pairs = I.visible_pairs(wl.S, wl.T, wl.visibility, wl.ratio, wl.q_pos0)
+    value = pairs * world / (ms_step * 1e-3) / 1e9
+    peak_mem = torch.cuda.max_memory_allocated(dev) / 1e9
+
+    pk = _peaks()
+    tensor_peak = pk["bf16"] * (2.0 if wl.dtype == "fp8" else 1.0)
+    kern_ms = statistics.mean(per)
+    achieved = pairs * flops_per_pair(wl) / (kern_ms * 1e-3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+        dbuf = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in host.items()}
+        h_idx = torch.empty(bufs[0].shape, dtype=torch.int32).pin_memory()
+        h_len = torch.empty(bufs[1].shape, dtype=torch.int32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+        d2h = h_idx.numel() * 4 + h_len.numel() * 4
+
+        def e2e_step():
+            for k_, v in host.items():
+                if v is not None:
+                    dbuf[k_].copy_(v, non_blocking=True)
+            I.topk(dbuf["q"], dbuf["k"], dbuf["w"], wl.K, visibility=wl.visibility, ratio=wl.ratio,
+                   q_pos0=wl.q_pos0, q_scale=dbuf["q_scale"], k_scale=dbuf["k_scale"],
+                   pool_coef=dbuf["pool_coef"], buffers=bufs, stream=stream)
+            h_idx.copy_(bufs[0], non_blocking=True)
+            h_len.copy_(bufs[1], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n_e2e = max(1, min(args.steps, 5))
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        e2e = {"value": pairs * world / (e2e_ms * 1e-3) / 1e9, "unit": "Gpairs/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        del host, dbuf
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(wl)
+
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            traffic = json.load(f).get(wl.name)
+    except Exception:
+        traffic = None
+
+    launches_per_step = 1 + (1 if wl.visibility == W.POOLED else 0)
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "Gpairs/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8-e4m3 (fp32 accumulate)" if wl.dtype == "fp8" else "bf16 (fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "S": wl.S, "T": wl.T, "H": wl.H, "D": wl.D, "K": wl.K,
+                       "visibility": ["token", "compressed", "pooled"][wl.visibility], "ratio": wl.ratio,
+                       "q_pos0": wl.q_pos0, "parallelism": f"{world} independent problems (one per GPU)",
+                       "l2": "inputs larger than L2 (q alone is "
+                             f"{inp['q'].numel() * inp['q'].element_size() / 2**30:.2f} GiB)"},
+            "pairs_per_step": pairs, "queries_per_s": wl.S * world / (ms_step * 1e-3),
+            "tensor_peak_frac": achieved / tensor_peak,
+            "peak_hbm_gb": peak_mem,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                         "frac": achieved / tensor_peak, "traffic": traffic,
+                         "peak_source": f"{pk['source']} bf16 burst" + (" x2 for fp8 (nominal ratio)" if wl.dtype == "fp8" else ""),
+                         "flops_per_pair": flops_per_pair(wl)},
+            "clocks": clk.summary(),
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "device_status": status,
+            "cpu_baseline": base,
+        }
+        print(json.dumps(out))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

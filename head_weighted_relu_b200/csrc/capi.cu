@@ -1,0 +1,273 @@
+// capi.cu -- host runtime behind include/hwr_indexer.h: argument checks,
+// workspace carving, TMA descriptors and launches on the caller's stream.
+// Nothing here allocates device memory or synchronises (except
+// indexer_read_status, which says so).
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "../../include/hwr_indexer.h"
+#include "internal.h"
+
+namespace hwr {
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+constexpr int kMaxDevices = 64;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool sm100 = false;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+indexer_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return INDEXER_ECUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (g_dev[dev].sms == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return INDEXER_ECUDA;
+    g_dev[dev].sms = sms;
+    g_dev[dev].sm100 = (major == 10 && minor == 0);
+  }
+  *out = g_dev[dev];
+  return INDEXER_OK;
+}
+
+// Everything derived from a validated problem.
+struct Plan {
+  ScoreVariant var;
+  int64_t n_keys;    // rows scored: T, or T / ratio pools
+  int32_t ksel;      // keys (pools) selected per query
+  int32_t width;     // output row width
+  int32_t out_ratio;
+  int32_t ranged;
+  int32_t n_blocks;
+  int32_t grid;
+  int32_t cap;
+  size_t kp_bytes;   // pooled keys (POOLED only)
+  size_t cand_bytes;
+  size_t ws_bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
+  if (!p) return INDEXER_EINVAL;
+  if (p->S < 0 || p->T < 1 || p->q_pos0 < 0 || p->K < 1 || p->flags != 0 || p->reserved != 0)
+    return INDEXER_EINVAL;
+  if (p->visibility < INDEXER_VIS_TOKEN || p->visibility > INDEXER_VIS_POOLED) return INDEXER_EINVAL;
+  if (p->dtype != INDEXER_BF16 && p->dtype != INDEXER_FP8_E4M3) return INDEXER_EINVAL;
+  if (p->S > (int64_t(1) << 31) / 64 || p->T > (int64_t(1) << 30) || p->q_pos0 > (int64_t(1) << 40))
+    return INDEXER_EUNSUPPORTED;
+  const bool token = p->visibility == INDEXER_VIS_TOKEN;
+  const int ratio = token ? 1 : p->ratio;
+  if (!token && (ratio < 1 || ratio > 16)) return INDEXER_EINVAL;
+  if (p->visibility != INDEXER_VIS_COMPRESSED && p->q_pos0 + p->S > p->T) return INDEXER_EINVAL;
+  if (p->visibility == INDEXER_VIS_POOLED) {
+    if (p->K % ratio != 0) return INDEXER_EINVAL;
+    if (p->dtype != INDEXER_BF16) return INDEXER_EUNSUPPORTED;
+  }
+  if (!score_variant(p->H, p->D, p->dtype == INDEXER_FP8_E4M3, &pl->var)) return INDEXER_EUNSUPPORTED;
+  pl->n_keys = p->visibility == INDEXER_VIS_POOLED ? p->T / ratio : p->T;
+  pl->ksel = p->visibility == INDEXER_VIS_POOLED ? p->K / ratio : p->K;
+  if (pl->ksel > (1 << 20)) return INDEXER_EUNSUPPORTED;
+  pl->width = p->visibility == INDEXER_VIS_POOLED ? p->K + ratio - 1 : p->K;
+  pl->out_ratio = p->visibility == INDEXER_VIS_POOLED ? ratio : 1;
+  pl->ranged = token ? 0 : 1;
+  const int64_t nb = (p->S + pl->var.queries_per_block - 1) / pl->var.queries_per_block;
+  pl->n_blocks = static_cast<int32_t>(nb);
+  pl->cap = candidate_capacity(pl->ksel);
+  pl->grid = 0;
+  pl->cand_bytes = 0;
+  if (need_device) {
+    DeviceInfo di;
+    const indexer_status st = device_info(&di);
+    if (st != INDEXER_OK) return st;
+    pl->grid = static_cast<int32_t>(nb < di.sms ? nb : di.sms);
+    pl->cand_bytes = static_cast<size_t>(pl->grid) * 2 * pl->var.queries_per_wg * static_cast<size_t>(pl->cap) *
+                     sizeof(uint2);
+  }
+  pl->kp_bytes = p->visibility == INDEXER_VIS_POOLED
+                     ? align256(static_cast<size_t>(pl->n_keys) * p->D * 2)
+                     : 0;
+  pl->ws_bytes = kStatusBytes + pl->kp_bytes + align256(pl->cand_bytes);
+  return INDEXER_OK;
+}
+
+bool encode_2d(CUtensorMap* tm, const void* base, bool fp8, int64_t rows, int D, int box_rows) {
+  const int elem = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * elem};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(tm, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+}  // namespace hwr
+
+using namespace hwr;
+
+extern "C" {
+
+int32_t indexer_abi_version(void) { return 1; }
+
+const char* indexer_status_string(indexer_status s) {
+  switch (s) {
+    case INDEXER_OK: return "ok";
+    case INDEXER_EINVAL: return "invalid argument";
+    case INDEXER_EWORKSPACE: return "workspace missing, misaligned or too small";
+    case INDEXER_EUNSUPPORTED: return "problem outside the compiled variants";
+    case INDEXER_ECUDA: return "CUDA call failed";
+    case INDEXER_EDEVICE: return "device is not sm_100 (B200 class)";
+  }
+  return "unknown status";
+}
+
+indexer_status indexer_out_width(const indexer_problem* p, int32_t* width) {
+  Plan pl;
+  const indexer_status st = make_plan(p, false, &pl);
+  if (st != INDEXER_OK) return st;
+  if (!width) return INDEXER_EINVAL;
+  *width = pl.width;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_workspace_bytes(const indexer_problem* p, size_t* bytes) {
+  Plan pl;
+  const indexer_status st = make_plan(p, true, &pl);
+  if (st != INDEXER_OK) return st;
+  if (!bytes) return INDEXER_EINVAL;
+  *bytes = pl.ws_bytes;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_topk(const indexer_problem* p, const void* q, const void* k, const float* w,
+                            const float* q_scale, const float* k_scale, const void* pool_coef, int32_t* out_idx,
+                            int32_t* out_len, float* out_score, void* workspace, size_t workspace_bytes,
+                            void* stream_) {
+  Plan pl;
+  indexer_status st = make_plan(p, true, &pl);
+  if (st != INDEXER_OK) return st;
+  DeviceInfo di;
+  st = device_info(&di);
+  if (st != INDEXER_OK) return st;
+  if (!di.sm100) return INDEXER_EDEVICE;
+  const bool fp8 = p->dtype == INDEXER_FP8_E4M3;
+  const bool pooled = p->visibility == INDEXER_VIS_POOLED;
+  if (p->S > 0 && (!q || !w || !out_idx || !out_len)) return INDEXER_EINVAL;
+  if (!k || !aligned(k, 16) || (q && !aligned(q, 16))) return INDEXER_EINVAL;
+  if (fp8 && (!q_scale || !k_scale)) return INDEXER_EINVAL;
+  if (pooled && !pool_coef) return INDEXER_EINVAL;
+  if (!workspace || !aligned(workspace, 256)) return INDEXER_EWORKSPACE;
+  if (workspace_bytes < pl.ws_bytes) return INDEXER_EWORKSPACE;
+  if (!get_encoder()) return INDEXER_ECUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  void* kp = ws + kStatusBytes;
+  uint2* cand = reinterpret_cast<uint2*>(ws + kStatusBytes + pl.kp_bytes);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), stream) != cudaSuccess) return INDEXER_ECUDA;
+  if (p->S == 0) return INDEXER_OK;
+
+  const void* keys = k;
+  if (pooled) {
+    if (launch_pool_keys(k, pl.n_keys, p->D, pool_coef, p->ratio, kp, stream) != cudaSuccess)
+      return INDEXER_ECUDA;
+    keys = kp;
+  }
+
+  CUtensorMap tm_q, tm_k;
+  if (!encode_2d(&tm_q, q, fp8, p->S * p->H, p->D, pl.var.q_box_rows)) return INDEXER_ECUDA;
+  if (!encode_2d(&tm_k, keys, fp8, pl.n_keys, p->D, 128)) return INDEXER_ECUDA;
+
+  ScoreParams sp;
+  sp.S = p->S;
+  sp.n_keys = pl.n_keys;
+  sp.q_pos0 = p->q_pos0;
+  sp.ranged = pl.ranged;
+  sp.ratio = pl.ranged ? p->ratio : 1;
+  sp.out_ratio = pl.out_ratio;
+  sp.ksel = pl.ksel;
+  sp.width = pl.width;
+  sp.n_blocks = pl.n_blocks;
+  sp.cap = pl.cap;
+  sp.w = w;
+  sp.q_scale = q_scale;
+  sp.k_scale = k_scale;
+  sp.out_idx = out_idx;
+  sp.out_len = out_len;
+  sp.out_score = out_score;
+  sp.cand = cand;
+  sp.status = status;
+
+  if (cudaFuncSetAttribute(pl.var.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.var.smem_bytes) !=
+      cudaSuccess)
+    return INDEXER_ECUDA;
+  void* args[] = {&tm_q, &tm_k, &sp};
+  if (cudaLaunchKernel(pl.var.fn, dim3(pl.grid), dim3(pl.var.threads), args, pl.var.smem_bytes, stream) !=
+      cudaSuccess)
+    return INDEXER_ECUDA;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_pool_keys(const void* k, int64_t T_tokens, int32_t D, const void* pool_coef,
+                                 int32_t ratio, void* out_kp, void* stream) {
+  if (!k || !pool_coef || !out_kp || T_tokens < 0 || D < 1 || D > 4096 || ratio < 1 || ratio > 16)
+    return INDEXER_EINVAL;
+  if (launch_pool_keys(k, T_tokens / ratio, D, pool_coef, ratio, out_kp, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return INDEXER_ECUDA;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_pair_overlap(const int32_t* idx, const int32_t* len, int64_t S, int32_t width,
+                                    int32_t* out_shared, void* stream) {
+  if (S < 0 || width < 0) return INDEXER_EINVAL;
+  if (S / 2 == 0) return INDEXER_OK;
+  if (!idx || !len || !out_shared) return INDEXER_EINVAL;
+  if (launch_pair_overlap(idx, len, S / 2, width, out_shared, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return INDEXER_ECUDA;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_read_status(void* workspace, int32_t* flags, void* stream) {
+  if (!workspace || !flags) return INDEXER_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return INDEXER_ECUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return INDEXER_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return INDEXER_ECUDA;
+  *flags = static_cast<int32_t>(v);
+  return INDEXER_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// internal.h -- declarations shared by the host runtime and the kernels of
+// the indexer library (not part of the public C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hwr {
+
+// Device status bits kept in the first word of the workspace.
+constexpr uint32_t kStatusWaitTimeout = 1u;
+constexpr uint32_t kStatusOverflow = 2u;
+
+// Arguments of the scoring + top-K kernel (one launch per indexer call).
+struct ScoreParams {
+  int64_t S;          // query rows
+  int64_t n_keys;     // rows of the scored key matrix (tokens, compressed keys or pools)
+  int64_t q_pos0;     // global position of query row 0
+  int32_t ranged;     // 0: key i visible iff i <= g; 1: key j visible iff ratio*j + ratio - 1 <= g
+  int32_t ratio;      // key span for ranged visibility
+  int32_t out_ratio;  // 1, or the pool width: each selected pool expands to out_ratio positions + tail
+  int32_t ksel;       // keys (pools) to select per query
+  int32_t width;      // row stride of out_idx / out_score
+  int32_t n_blocks;   // query blocks
+  int32_t cap;        // candidate-buffer entries per query
+  const float* w;        // [S, H]
+  const float* q_scale;  // [S, H] or null (FP8)
+  const float* k_scale;  // [n_keys] or null (FP8)
+  int32_t* out_idx;      // [S, width]
+  int32_t* out_len;      // [S]
+  float* out_score;      // [S, width] or null
+  uint2* cand;           // candidate buffers: [grid][2][queries per warpgroup][cap]
+  uint32_t* status;      // device status word
+};
+
+// Per-variant launch facts, filled by the kernel's translation unit.
+struct ScoreVariant {
+  const void* fn;         // kernel function
+  int queries_per_block;  // QB
+  int queries_per_wg;     // NQA
+  int q_box_rows;         // rows of the q TMA box
+  int box_elems;          // inner extent of every TMA box (128 bytes)
+  int smem_bytes;         // dynamic shared memory
+  int threads;
+};
+
+// Returns false when (H, D, fp8) has no compiled variant.
+bool score_variant(int H, int D, bool fp8, ScoreVariant* out);
+
+// Candidate-buffer capacity per query for a selection budget of ksel keys.
+inline int candidate_capacity(int ksel) {
+  int c = ((2 * ksel + 127) / 128) * 128 + 128;
+  return c;
+}
+
+cudaError_t launch_pool_keys(const void* k, int64_t n_pools, int D, const void* coef, int ratio, void* out,
+                             cudaStream_t stream);
+cudaError_t launch_pair_overlap(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
+                                int32_t* out, cudaStream_t stream);
+
+}  // namespace hwr

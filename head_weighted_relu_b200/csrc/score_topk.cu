@@ -1,0 +1,664 @@
+// score_topk.cu -- the indexer's hot path on sm_100a: tcgen05 scoring with the
+// ReLU / signed head weights / visibility mask fused into the TMEM epilogue,
+// and a streaming exact top-K per query.  Scores are never written to HBM.
+//
+// Method ("DoSA: Dots Sparse Attention", section 前置知识 / background):
+//   s[t,i] = sum_h w[t,h] * max(0, q[t,h,:] . k[i,:])
+// for every key i visible to query t, then the K best keys of each query
+// (higher score first, then lower key index), emitted in key order with a
+// valid length ("Adjacent-Query KV-Index Overlap in 256K DSA Training", §3).
+// StreamIndex (arXiv 2605.02568, abstract) streams keys through a chunked
+// partition-merge top-K instead of materialising scores; this kernel streams
+// keys in ascending order and merges into a running selection.
+//
+// One persistent CTA per SM, 10 warps:
+//   warp 0      TMA producer: the query block's q rows once, then key tiles of
+//               128 rows through a ring of shared-memory stages;
+//   warp 1      MMA issuer: for each key tile, two accumulators
+//               acc[a][key, (query, head)] = k_tile . q_block[a]^T
+//               (M = 128 keys = TMEM lanes, N = queries x heads <= 256 columns,
+//               K = D), tcgen05.mma with FP32 accumulation in TMEM;
+//   warps 2..9  two epilogue warpgroups, one per accumulator.  Each thread owns
+//               one key (one TMEM lane) and, for every query of its group,
+//               reduces sum_h w[t,h] * max(acc, 0) in registers, applies the
+//               visibility mask, and appends (ordered score, key) pairs that
+//               beat the query's running threshold to a per-query candidate
+//               buffer in global memory -- in key order, so the buffer is
+//               always sorted by key index.  A buffer about to overflow is cut
+//               back to its exact top-K by a warpgroup radix select, which
+//               raises the threshold.  After the query block's last tile the
+//               same select gives the final top-K, written in key order.
+//
+// Keys arrive in ascending index order, so once a buffer holds the top-K of
+// the keys seen so far with K-th entry (v, i), a later key (index > i) can
+// only enter the final top-K with a score strictly above v: the threshold is
+// exact for the tie rule, and every candidate the final select sees is kept
+// or rejected exactly as a full sort of the score row would.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace hwr {
+
+constexpr int kThreads = 320;
+constexpr int kBM = 128;                         // keys per tile = MMA M = TMEM lanes
+constexpr int kHistBins = 2048;                  // 11-bit radix digits
+constexpr int kSmemLimit = 232448;               // 227 KB opt-in shared memory per CTA
+constexpr uint64_t kWaitLimitNs = 4000000000ull; // give up a pipeline wait after 4 s
+
+template <int NQA>
+struct WgState {
+  uint32_t thr[NQA];     // a candidate is appended iff its ordered score >= thr
+  int32_t cnt[2][NQA];   // candidates held, double-buffered by tile parity
+  int32_t nvis[NQA];     // keys visible to each query of the group
+  int32_t wc[NQA][4];    // per-warp pass counts of the current tile
+  uint32_t red[16];      // reduction scratch
+  int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
+};
+
+template <int STAGES>
+struct Barriers {
+  uint64_t kfull[STAGES];
+  uint64_t kempty[STAGES];
+  uint64_t qfull, qempty;
+  uint64_t accfull[2], accempty[2];
+  uint64_t mma_done;
+  uint32_t tmem_slot;
+  int abort;
+};
+
+template <int H, int D, bool FP8>
+struct Cfg {
+  static constexpr int ELEM = FP8 ? 1 : 2;
+  static constexpr int ROW_BYTES = D * ELEM;
+  static constexpr int NBOX = ROW_BYTES / 128;          // 128-byte swizzle boxes per row
+  static constexpr int BOX_ELEMS = 128 / ELEM;
+  static constexpr int KSTEPS = ROW_BYTES / 32;          // MMA K steps of 32 bytes
+  static constexpr int NQA = (256 / H) < 16 ? (256 / H) : 16;  // queries per accumulator
+  static constexpr int BN = NQA * H;                     // accumulator columns = MMA N
+  static constexpr int QB = 2 * NQA;                     // queries per block
+  static constexpr int CHUNKS = BN / 64;                 // 64-column TMEM loads per accumulator
+  static constexpr int QPC = 64 / H;                     // queries per 64-column load
+  static constexpr int Q_ACC_BYTES = BN * ROW_BYTES;
+  static constexpr int Q_BYTES = 2 * Q_ACC_BYTES;
+  static constexpr int K_STAGE_BYTES = kBM * ROW_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMALL_BYTES = kHistBins * 4 * 2 + 2 * BN * 4 + 2 * (int)sizeof(WgState<NQA>);
+  static constexpr int AVAIL = kSmemLimit - 1024 - Q_BYTES - SMALL_BYTES - (int)sizeof(Barriers<8>);
+  static constexpr int STAGES_RAW = AVAIL / K_STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_HIST = OFF_K + STAGES * K_STAGE_BYTES;
+  static constexpr int OFF_W = OFF_HIST + kHistBins * 4 * 2;
+  static constexpr int OFF_ST = OFF_W + 2 * BN * 4;
+  static constexpr int OFF_BAR = OFF_ST + 2 * (int)sizeof(WgState<NQA>);
+  static constexpr int SMEM_BYTES = 1024 + OFF_BAR + (int)sizeof(Barriers<STAGES>);
+  static constexpr uint32_t IDESC = FP8 ? idesc_e4m3<kBM, BN>() : idesc_bf16<kBM, BN>();
+  static_assert(H % 4 == 0 && H <= 64, "heads");
+  static_assert(ROW_BYTES % 128 == 0, "row must be whole 128-byte swizzle rows");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "accumulator width");
+  static_assert(STAGES >= 2, "shared memory too small for a 2-stage key ring");
+  static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
+  static_assert(OFF_K % 1024 == 0 && K_STAGE_BYTES % 1024 == 0 && Q_ACC_BYTES % 1024 == 0, "swizzle alignment");
+  static_assert(OFF_BAR % 8 == 0 && OFF_ST % 16 == 0 && OFF_W % 16 == 0, "alignment");
+};
+
+__device__ __forceinline__ int32_t n_visible(const ScoreParams& p, int64_t g) {
+  const int64_t n = p.ranged ? (g + 1) / p.ratio : g + 1;
+  return static_cast<int32_t>(n < p.n_keys ? n : p.n_keys);
+}
+
+// Heaviest query blocks first (they see the most keys), dealt to the CTAs in
+// a snake order so that per-CTA work evens out.  -1 once this CTA is done.
+__device__ __forceinline__ int block_of(int round, int cta, int grid, int n_blocks) {
+  const int item = round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+  return item < n_blocks ? n_blocks - 1 - item : -1;
+}
+
+template <int QB>
+__device__ __forceinline__ int tiles_of_block(const ScoreParams& p, int b) {
+  int64_t t_last = static_cast<int64_t>(b + 1) * QB - 1;
+  if (t_last >= p.S) t_last = p.S - 1;
+  const int32_t n = n_visible(p, p.q_pos0 + t_last);
+  return (n + kBM - 1) / kBM;
+}
+
+template <int H, int QPC>
+__device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float* w, float* s) {
+#pragma unroll
+  for (int qq = 0; qq < QPC; ++qq) {
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int h = 0; h < H; h += 4) {
+      const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
+      a0 = fmaf(wv.x, fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f), a0);
+      a1 = fmaf(wv.y, fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f), a1);
+      a0 = fmaf(wv.z, fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f), a0);
+      a1 = fmaf(wv.w, fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f), a1);
+    }
+    s[qq] = a0 + a1;
+  }
+}
+
+// ------------------------------------------------------------------------
+// Warpgroup-cooperative selection over a candidate buffer (128 threads).
+// ------------------------------------------------------------------------
+struct SelResult {
+  uint32_t v;      // the rank-th largest value
+  uint32_t above;  // entries (passing the filter) with a larger value
+  uint32_t eq;     // entries equal to v
+};
+
+// rank-th largest (1-based) of f(e) over buf[0, n), where f(e) = e.x (ordered
+// score) or ~e.y (so that the largest is the lowest index), counting only the
+// entries with e.x == fval when `filt`.  `total` = entries passing the filter.
+// MSB-first radix select with 11-bit digits, starting below the bits that all
+// entries share.
+__device__ SelResult wg_radix_select(const uint2* buf, int n, uint32_t rank, bool idx_field, bool filt,
+                                     uint32_t fval, uint32_t total, uint32_t* hist, uint32_t* red,
+                                     int etid, int bar_id) {
+  const int lane = etid & 31, wq = etid >> 5;
+  uint32_t mx = 0u, mn = 0xFFFFFFFFu;
+  for (int i = etid; i < n; i += kBM) {
+    const uint2 e = buf[i];
+    if (!filt || e.x == fval) {
+      const uint32_t f = idx_field ? ~e.y : e.x;
+      mx = max(mx, f);
+      mn = min(mn, f);
+    }
+  }
+  mx = warp_max_u32(mx);
+  mn = warp_min_u32(mn);
+  if (lane == 0) {
+    red[wq] = mx;
+    red[4 + wq] = mn;
+  }
+  named_bar(bar_id, kBM);
+  mx = max(max(red[0], red[1]), max(red[2], red[3]));
+  mn = min(min(red[4], red[5]), min(red[6], red[7]));
+  named_bar(bar_id, kBM);
+  if (mx == mn) return {mx, 0u, total};
+  int lo = 32 - __clz(mx ^ mn);  // bits [lo, 32) are shared by every entry
+  uint32_t prefix = lo >= 32 ? 0u : (mx >> lo) << lo;
+  uint32_t rem = rank, above = 0u, eq = 0u;
+  while (lo > 0) {
+    const int width = lo < 11 ? lo : 11;
+    const int shift = lo - width;
+    const int nb = 1 << width;
+    for (int i = etid; i < nb; i += kBM) hist[i] = 0u;
+    named_bar(bar_id, kBM);
+    for (int i = etid; i < n; i += kBM) {
+      const uint2 e = buf[i];
+      if (filt && e.x != fval) continue;
+      const uint32_t f = idx_field ? ~e.y : e.x;
+      if (lo < 32 && (f >> lo) != (prefix >> lo)) continue;
+      atomicAdd(&hist[(f >> shift) & static_cast<uint32_t>(nb - 1)], 1u);
+    }
+    named_bar(bar_id, kBM);
+    // thread etid owns bins [b0, b1); ranks count from the top bin down
+    const int per = nb >= kBM ? nb / kBM : 1;
+    const int b0 = etid * per;
+    const int b1 = min(b0 + per, nb);
+    uint32_t local = 0u;
+    for (int b = b0; b < b1; ++b) local += hist[b];
+    uint32_t incl = local;  // sum over lanes >= this lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(kFullMask, incl, o);
+      if (lane + o < 32) incl += t;
+    }
+    if (lane == 0) red[wq] = incl;
+    named_bar(bar_id, kBM);
+    uint32_t higher = 0u;
+    for (int w2 = wq + 1; w2 < 4; ++w2) higher += red[w2];
+    const uint32_t excl = incl - local + higher;  // entries in bins owned by higher threads
+    if (local > 0u && excl < rem && rem <= excl + local) {
+      uint32_t acc = excl;
+      for (int b = b1 - 1; b >= b0; --b) {
+        const uint32_t h = hist[b];
+        if (acc + h >= rem) {
+          red[8] = static_cast<uint32_t>(b);
+          red[9] = acc;  // entries above digit b in this pass
+          red[10] = h;
+          break;
+        }
+        acc += h;
+      }
+    }
+    named_bar(bar_id, kBM);
+    const uint32_t d = red[8];
+    rem -= red[9];
+    above += red[9];
+    eq = red[10];
+    prefix |= d << shift;
+    lo = shift;
+    named_bar(bar_id, kBM);
+  }
+  return {prefix, above, eq};
+}
+
+// Entries to keep: e.x > v, or e.x == v and e.y <= icut.
+struct Cut {
+  uint32_t v;
+  uint32_t icut;
+};
+
+// Exact top-`ksel` of buf[0, n) under (higher ordered score, then lower index).
+__device__ Cut wg_topk_cut(const uint2* buf, int n, uint32_t ksel, uint32_t* hist, uint32_t* red, int etid,
+                           int bar_id) {
+  const SelResult s1 = wg_radix_select(buf, n, ksel, false, false, 0u, static_cast<uint32_t>(n), hist, red,
+                                       etid, bar_id);
+  const uint32_t need = ksel - s1.above;  // entries equal to v that make the cut
+  if (need >= s1.eq) return {s1.v, 0xFFFFFFFFu};
+  // the need-th lowest index among the entries tied at v
+  const SelResult s2 = wg_radix_select(buf, n, need, true, true, s1.v, s1.eq, hist, red, etid, bar_id);
+  return {s1.v, ~s2.v};
+}
+
+// Streams buf[0, n) in order and calls emit(pos, e) for every kept entry, pos
+// counting kept entries in buffer order.  In place (emit writing buf[pos]) is
+// safe: pos never exceeds the entry's own index and reads of a chunk finish
+// before its writes.  Returns the number kept.
+template <class Emit>
+__device__ int wg_compact(const uint2* buf, int n, Cut c, bool keep_all, int32_t* cwc, int etid, int bar_id,
+                          Emit emit) {
+  const int lane = etid & 31, wq = etid >> 5;
+  int running = 0, par = 0;
+  for (int base = 0; base < n; base += kBM) {
+    const int i = base + etid;
+    uint2 e = make_uint2(0u, 0u);
+    bool keep = false;
+    if (i < n) {
+      e = buf[i];
+      keep = keep_all || e.x > c.v || (e.x == c.v && e.y <= c.icut);
+    }
+    const uint32_t bal = __ballot_sync(kFullMask, keep);
+    if (lane == 0) cwc[par * 4 + wq] = __popc(bal);
+    named_bar(bar_id, kBM);
+    int prior = 0, tot = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < 4; ++w2) {
+      const int cc = cwc[par * 4 + w2];
+      tot += cc;
+      prior += (w2 < wq) ? cc : 0;
+    }
+    if (keep) emit(running + prior + __popc(bal & ((1u << lane) - 1u)), e);
+    running += tot;
+    par ^= 1;
+  }
+  named_bar(bar_id, kBM);
+  return running;
+}
+
+// ------------------------------------------------------------------------
+// The kernel.
+// ------------------------------------------------------------------------
+template <int H, int D, bool FP8>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const ScoreParams p) {
+  using C = Cfg<H, D, FP8>;
+  constexpr int NQA = C::NQA;
+  constexpr int BN = C::BN;
+  constexpr int QB = C::QB;
+  constexpr int STAGES = C::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* hist_base = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
+  float* wsm_base = reinterpret_cast<float*>(smem + C::OFF_W);
+  WgState<NQA>* states = reinterpret_cast<WgState<NQA>*>(smem + C::OFF_ST);
+  Barriers<STAGES>* bars = reinterpret_cast<Barriers<STAGES>*>(smem + C::OFF_BAR);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bars->kfull[s], 1);
+      mbar_init(&bars->kempty[s], 1);
+    }
+    mbar_init(&bars->qfull, 1);
+    mbar_init(&bars->qempty, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->accfull[a], 1);
+      mbar_init(&bars->accempty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_slot;
+  volatile int* abort_flag = &bars->abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      int stage = 0;
+      uint32_t kph = 0, qe_ph = 0;
+      bool first = true, ok = true;
+      for (int r = 0; ok; ++r) {
+        const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
+        if (b < 0) break;
+        const int nt = tiles_of_block<QB>(p, b);
+        if (nt == 0) continue;
+        if (!first) {
+          ok = mbar_wait(&bars->qempty, qe_ph, abort_flag, kWaitLimitNs);
+          qe_ph ^= 1;
+          if (!ok) break;
+        }
+        first = false;
+        mbar_arrive_expect_tx(&bars->qfull, C::Q_BYTES);
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_2d(smem + C::OFF_Q + a * C::Q_ACC_BYTES + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS,
+                        (b * QB + a * NQA) * H, &bars->qfull);
+        for (int j = 0; j < nt; ++j) {
+          ok = mbar_wait(&bars->kempty[stage], kph ^ 1u, abort_flag, kWaitLimitNs);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars->kfull[stage], C::K_STAGE_BYTES);
+#pragma unroll
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_2d(smem + C::OFF_K + stage * C::K_STAGE_BYTES + bx * kBM * 128, &tm_k, bx * C::BOX_ELEMS,
+                        j * kBM, &bars->kfull[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            kph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        atomicOr(p.status, kStatusWaitTimeout);
+        bars->abort = 1;
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(smem + C::OFF_Q);
+      const uint32_t k_base = smem_u32(smem + C::OFF_K);
+      int stage = 0;
+      uint32_t kph = 0, qf_ph = 0;
+      uint32_t ae_ph[2] = {0u, 0u};
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
+        if (b < 0) break;
+        const int nt = tiles_of_block<QB>(p, b);
+        if (nt == 0) continue;
+        ok = mbar_wait(&bars->qfull, qf_ph, abort_flag, kWaitLimitNs);
+        qf_ph ^= 1u;
+        if (!ok) break;
+        for (int j = 0; j < nt && ok; ++j) {
+          ok = mbar_wait(&bars->kfull[stage], kph, abort_flag, kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kst = k_base + stage * C::K_STAGE_BYTES;
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            ok = mbar_wait(&bars->accempty[a], ae_ph[a] ^ 1u, abort_flag, kWaitLimitNs);
+            ae_ph[a] ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t qa = q_base + a * C::Q_ACC_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < C::KSTEPS; ++kk) {
+              const uint64_t adesc = sw128_desc(kst + (kk >> 2) * (kBM * 128) + (kk & 3) * 32);
+              const uint64_t bdesc = sw128_desc(qa + (kk >> 2) * (BN * 128) + (kk & 3) * 32);
+              if constexpr (FP8)
+                tc_mma_e4m3(tmem_base + a * BN, adesc, bdesc, C::IDESC, kk > 0 ? 1u : 0u);
+              else
+                tc_mma_bf16(tmem_base + a * BN, adesc, bdesc, C::IDESC, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars->accfull[a]);
+          }
+          if (!ok) break;
+          tc_commit(&bars->kempty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            kph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&bars->qempty);
+      }
+      if (!ok) {
+        atomicOr(p.status, kStatusWaitTimeout);
+        bars->abort = 1;
+      }
+      // all MMAs issued by this thread have completed before TMEM is freed
+      tc_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0u, abort_flag, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------ epilogue warpgroups
+    const int wg = (warp - 2) >> 2;
+    const int wq = warp & 3;           // TMEM lane quarter accessible to this warp
+    const int etid = wq * 32 + lane;   // key row within the tile == order within the group
+    const int bar_id = 1 + wg;
+    WgState<NQA>* st = states + wg;
+    float* wsm = wsm_base + wg * BN;
+    uint32_t* hist = hist_base + wg * kHistBins;
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(wg * BN);
+    uint32_t af_ph = 0u;
+    int par = 0;
+    bool failed = false;
+    for (int r = 0; !failed; ++r) {
+      const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
+      if (b < 0) break;
+      const int nt = tiles_of_block<QB>(p, b);
+      const int64_t tq0 = static_cast<int64_t>(b) * QB + wg * NQA;
+      uint2* cand = p.cand + (static_cast<size_t>(blockIdx.x) * 2 + wg) * NQA * static_cast<size_t>(p.cap);
+
+      named_bar(bar_id, kBM);  // the previous block is completely done with the state
+      for (int i = etid; i < BN; i += kBM) {
+        const int64_t t = tq0 + i / H;
+        float v = 0.f;
+        if (t < p.S) {
+          v = p.w[t * H + (i % H)];
+          if constexpr (FP8) v *= p.q_scale[t * H + (i % H)];
+        }
+        wsm[i] = v;
+      }
+      if (etid < NQA) {
+        const int64_t t = tq0 + etid;
+        st->nvis[etid] = t < p.S ? n_visible(p, p.q_pos0 + t) : 0;
+        st->cnt[par][etid] = 0;
+        st->thr[etid] = 0u;
+      }
+      named_bar(bar_id, kBM);
+
+      for (int j = 0; j < nt; ++j) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&bars->accfull[wg], af_ph, abort_flag, kWaitLimitNs);
+        ok = __shfl_sync(kFullMask, ok ? 1 : 0, 0) != 0;
+        af_ph ^= 1u;
+        float s[NQA];
+#pragma unroll
+        for (int qi = 0; qi < NQA; ++qi) s[qi] = 0.f;
+        if (ok) {
+          tc_fence_after();
+          uint32_t ra[64], rb[64];
+          tmem_ld_x64(tbase, ra);
+          tmem_wait_ld(ra);
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            if ((c & 1) == 0) {
+              if (c + 1 < C::CHUNKS) tmem_ld_x64(tbase + (c + 1) * 64, rb);
+              score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
+              if (c + 1 < C::CHUNKS) tmem_wait_ld(rb);
+            } else {
+              if (c + 1 < C::CHUNKS) tmem_ld_x64(tbase + (c + 1) * 64, ra);
+              score_chunk<H, C::QPC>(rb, wsm + c * 64, s + c * C::QPC);
+              if (c + 1 < C::CHUNKS) tmem_wait_ld(ra);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->accempty[wg]);
+        }
+        const int32_t key = j * kBM + etid;
+        if constexpr (FP8) {
+          const float ks = key < p.n_keys ? p.k_scale[key] : 0.f;
+#pragma unroll
+          for (int qi = 0; qi < NQA; ++qi) s[qi] *= ks;
+        }
+        // pass flags and per-warp counts
+#pragma unroll
+        for (int qi = 0; qi < NQA; ++qi) {
+          const uint32_t okey = ordered_key(__fadd_rn(s[qi], 0.f));
+          const bool pass = ok && key < st->nvis[qi] && okey >= st->thr[qi];
+          const uint32_t bal = __ballot_sync(kFullMask, pass);
+          if (lane == 0) st->wc[qi][wq] = __popc(bal);
+        }
+        if (named_bar_or(bar_id, kBM, !ok)) {
+          failed = true;
+          break;
+        }
+        // ordered append: position = held + earlier warps + earlier lanes
+        const int np = par ^ 1;
+#pragma unroll
+        for (int qi = 0; qi < NQA; ++qi) {
+          const uint32_t okey = ordered_key(__fadd_rn(s[qi], 0.f));
+          const bool pass = key < st->nvis[qi] && okey >= st->thr[qi];
+          const uint32_t bal = __ballot_sync(kFullMask, pass);
+          const int held = st->cnt[par][qi];
+          int prior = 0, tot = 0;
+#pragma unroll
+          for (int w2 = 0; w2 < 4; ++w2) {
+            const int cc = st->wc[qi][w2];
+            tot += cc;
+            prior += (w2 < wq) ? cc : 0;
+          }
+          if (pass) {
+            const int pos = held + prior + __popc(bal & ((1u << lane) - 1u));
+            cand[qi * static_cast<size_t>(p.cap) + pos] = make_uint2(okey, static_cast<uint32_t>(key));
+          }
+          if (etid == qi) st->cnt[np][qi] = held + tot;
+        }
+        named_bar(bar_id, kBM);
+        par = np;
+        // cut buffers that could not take another full tile back to their top-K
+#pragma unroll 1
+        for (int qi = 0; qi < NQA; ++qi) {
+          const int n = st->cnt[par][qi];
+          if (n > p.cap - kBM) {
+            uint2* buf = cand + qi * static_cast<size_t>(p.cap);
+            const Cut cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
+            wg_compact(buf, n, cut, false, &st->cwc[0][0], etid, bar_id,
+                       [&](int pos, uint2 e) { buf[pos] = e; });
+            if (etid == 0) {
+              st->cnt[par][qi] = p.ksel;
+              st->thr[qi] = cut.v == 0xFFFFFFFFu ? cut.v : cut.v + 1u;
+            }
+            named_bar(bar_id, kBM);
+          }
+        }
+      }
+      if (failed) break;
+
+      // final selection of each query of the group, written in key order
+#pragma unroll 1
+      for (int qi = 0; qi < NQA; ++qi) {
+        const int64_t t = tq0 + qi;
+        if (t >= p.S) continue;
+        const int n = st->cnt[par][qi];
+        uint2* buf = cand + qi * static_cast<size_t>(p.cap);
+        const bool all = n <= p.ksel;
+        Cut cut{0u, 0xFFFFFFFFu};
+        if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
+        int32_t* orow = p.out_idx + t * p.width;
+        float* srow = p.out_score ? p.out_score + t * p.width : nullptr;
+        const int m = p.out_ratio;
+        const int kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id, [&](int pos, uint2 e) {
+          const float sc = key_to_float(e.x);
+          if (m == 1) {
+            orow[pos] = static_cast<int32_t>(e.y);
+            if (srow) srow[pos] = sc;
+          } else {
+            for (int rr = 0; rr < m; ++rr) {
+              orow[pos * m + rr] = static_cast<int32_t>(e.y) * m + rr;
+              if (srow) srow[pos * m + rr] = sc;
+            }
+          }
+        });
+        int len = kept * m;
+        if (m > 1) {
+          const int64_t g = p.q_pos0 + t;
+          const int tail = static_cast<int>((g + 1) % m);
+          const int64_t first = g + 1 - tail;
+          for (int i = etid; i < tail; i += kBM) {
+            orow[len + i] = static_cast<int32_t>(first + i);
+            if (srow) srow[len + i] = __uint_as_float(0x7FC00000u);
+          }
+          len += tail;
+        }
+        for (int i = len + etid; i < p.width; i += kBM) {
+          orow[i] = -1;
+          if (srow) srow[i] = __uint_as_float(0x7FC00000u);
+        }
+        if (etid == 0) p.out_len[t] = len;
+      }
+    }
+    if (failed && etid == 0) {
+      atomicOr(p.status, kStatusWaitTimeout);
+      bars->abort = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------
+// Variant table.
+// ------------------------------------------------------------------------
+template <int H, int D, bool FP8>
+static void fill_variant(ScoreVariant* v) {
+  using C = Cfg<H, D, FP8>;
+  v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8>);
+  v->queries_per_block = C::QB;
+  v->queries_per_wg = C::NQA;
+  v->q_box_rows = C::BN;
+  v->box_elems = C::BOX_ELEMS;
+  v->smem_bytes = C::SMEM_BYTES;
+  v->threads = kThreads;
+}
+
+bool score_variant(int H, int D, bool fp8, ScoreVariant* v) {
+#define HWR_VARIANT(h, d, f)           \
+  if (H == h && D == d && fp8 == f) { \
+    fill_variant<h, d, f>(v);          \
+    return true;                       \
+  }
+  HWR_VARIANT(4, 64, false)
+  HWR_VARIANT(4, 128, false)
+  HWR_VARIANT(8, 64, false)
+  HWR_VARIANT(8, 128, false)
+  HWR_VARIANT(16, 64, false)
+  HWR_VARIANT(16, 128, false)
+  HWR_VARIANT(32, 64, false)
+  HWR_VARIANT(32, 128, false)
+  HWR_VARIANT(64, 64, false)
+  HWR_VARIANT(64, 128, false)
+  HWR_VARIANT(16, 128, true)
+  HWR_VARIANT(32, 128, true)
+  HWR_VARIANT(64, 128, true)
+#undef HWR_VARIANT
+  return false;
+}
+
+}  // namespace hwr

@@ -1,0 +1,159 @@
+/*
+ * hwr_indexer.h -- C ABI of the B200 (sm_100a) DSA lightning indexer.
+ *
+ * The indexer scores, for every query t and every key i visible to it,
+ *
+ *     s[t,i] = sum_h  w[t,h] * max(0, q[t,h,:] . k[i,:])
+ *
+ * ("DoSA: Dots Sparse Attention", section 前置知识 / background: the indexer
+ * score with ReLU and head weights of either sign), keeps the K best keys of
+ * each query (ties: the higher score wins, then the lower key index; the same
+ * page, section 研究动机 / motivation, asks for exact top-K under one tie
+ * rule), and writes them sorted by key index with a valid length
+ * ("Adjacent-Query KV-Index Overlap in 256K DSA Training", §1 and §3).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named q, k, w, *_scale, pool_coef, out_*, workspace are DEVICE
+ *     pointers on the current CUDA device, owned by the caller; the library
+ *     never frees or retains them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Kernels are enqueued asynchronously on it; no call below
+ *     synchronises unless it says so.
+ *   - Argument errors are detected on the host before any launch and return a
+ *     status other than INDEXER_OK; nothing is launched then.
+ *   - The library allocates no device memory: scratch comes from the caller's
+ *     workspace (see indexer_workspace_bytes), so every launch is shape-stable
+ *     and can be replayed.
+ *   - Rows are row-major with the last dimension contiguous.
+ */
+#ifndef HWR_INDEXER_H
+#define HWR_INDEXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  INDEXER_OK = 0,
+  INDEXER_EINVAL = 1,        /* a size, pointer or enum is out of range      */
+  INDEXER_EWORKSPACE = 2,    /* workspace missing, misaligned or too small   */
+  INDEXER_EUNSUPPORTED = 3,  /* valid problem outside the compiled variants  */
+  INDEXER_ECUDA = 4,         /* a CUDA runtime / driver call failed          */
+  INDEXER_EDEVICE = 5        /* the device is not sm_100 (B200 class)        */
+} indexer_status;
+
+/* Which keys a query at global position g may see.
+ *   TOKEN:      token key i is visible iff i <= g ("Module 06 — DSA & KPool:
+ *               Selective Retrieval", §3: position i sees j iff j <= i).
+ *   COMPRESSED: key j summarises tokens m*j .. m*j+m-1 (m = `ratio`) and is
+ *               visible iff m*j + m - 1 <= g (StreamIndex, arXiv 2605.02568,
+ *               abstract: CSA keys compressed with m = 4; the completion rule
+ *               is KPool §3's).
+ *   POOLED:     k holds token keys; pool p is formed from tokens
+ *               m*p .. m*p+m-1 as kp[p] = RNE_bf16(sum_j c[j] (*) k[m*p+j])
+ *               (KPool §2: a channel-wise weighted representation of each
+ *               complete pool), is visible iff m*p + m - 1 <= g, the best
+ *               K/m pools are expanded to their m tokens, and the positions
+ *               of the query's own incomplete pool (m*floor((g+1)/m) .. g,
+ *               at most m-1) are appended as a tail (KPool §2). */
+typedef enum {
+  INDEXER_VIS_TOKEN = 0,
+  INDEXER_VIS_COMPRESSED = 1,
+  INDEXER_VIS_POOLED = 2
+} indexer_visibility;
+
+typedef enum {
+  INDEXER_BF16 = 0,      /* q, k in bfloat16                                  */
+  INDEXER_FP8_E4M3 = 1   /* q, k in FP8 e4m3 codes with FP32 per-row scales   */
+} indexer_dtype;
+
+typedef struct {
+  int64_t S;          /* query rows                                           */
+  int64_t T;          /* key rows: tokens (TOKEN, POOLED) or compressed keys  */
+  int32_t H;          /* indexer heads: 4, 8, 16, 32 or 64                    */
+  int32_t D;          /* head dim: 64 or 128 (BF16), 128 (FP8)                */
+  int64_t q_pos0;     /* global position of query row 0 (g = q_pos0 + t)      */
+  int32_t visibility; /* indexer_visibility                                   */
+  int32_t ratio;      /* m for COMPRESSED / POOLED (1..16); ignored for TOKEN */
+  int32_t K;          /* budget in positions; POOLED selects K/ratio pools    */
+  int32_t dtype;      /* indexer_dtype                                        */
+  int32_t flags;      /* must be 0                                            */
+  int32_t reserved;   /* must be 0                                            */
+} indexer_problem;
+
+/* Row width of out_idx / out_score: K, or K + ratio - 1 for POOLED (2,051 for
+ * K = 2,048 and pools of 4; KPool §2, "size index buffers to 2,051").
+ * Returns INDEXER_EINVAL for an invalid problem. */
+indexer_status indexer_out_width(const indexer_problem* p, int32_t* width);
+
+/* Bytes of device workspace indexer_topk needs for `p` on the CURRENT device
+ * (it depends on the device's SM count).  The workspace must be 256-byte
+ * aligned; its contents need no initialisation and are scratch between calls,
+ * except the status words read by indexer_read_status. */
+indexer_status indexer_workspace_bytes(const indexer_problem* p, size_t* bytes);
+
+/* The indexer: scores, top-K and finalisation in one call.
+ *   q         [S, H, D]  bf16, or e4m3 codes (uint8) for INDEXER_FP8_E4M3
+ *   k         [T, D]     same storage as q
+ *   w         [S, H]     float32 head weights (signed)
+ *   q_scale   [S, H]     float32, FP8 only (else NULL): q value = code*scale
+ *   k_scale   [T]        float32, FP8 only (else NULL): k value = code*scale
+ *   pool_coef [ratio, D] bf16, POOLED only (else NULL): the c[j] of kp
+ *   out_idx   [S, W]     int32, W = indexer_out_width: selected positions
+ *                        ascending, then -1 padding
+ *   out_len   [S]        int32 valid length of each row:
+ *                        min(K, visible) (TOKEN, COMPRESSED),
+ *                        ratio*min(K/ratio, pools) + tail (POOLED)
+ *   out_score [S, W]     float32 or NULL: the score of each selected entry in
+ *                        the same order (a pool's score for each of its
+ *                        tokens), NaN for tail and padding slots
+ *   workspace, workspace_bytes: scratch from the caller (see above)
+ * TOKEN and POOLED require q_pos0 + S <= T (every query has its own token).
+ * Asynchronous on `stream`; allocates nothing. */
+indexer_status indexer_topk(const indexer_problem* p,
+                            const void* q, const void* k, const float* w,
+                            const float* q_scale, const float* k_scale,
+                            const void* pool_coef,
+                            int32_t* out_idx, int32_t* out_len, float* out_score,
+                            void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Pool formation alone (the first step of POOLED):
+ *   kp[p, d] = RNE_bf16( exact sum_{j<ratio} c[j, d] * k[ratio*p + j, d] )
+ * for p < T_tokens / ratio; k [T_tokens, D] bf16, pool_coef [ratio, D] bf16,
+ * out_kp [T_tokens/ratio, D] bf16.  (KPool §2.) */
+indexer_status indexer_pool_keys(const void* k, int64_t T_tokens, int32_t D,
+                                 const void* pool_coef, int32_t ratio,
+                                 void* out_kp, void* stream);
+
+/* Exact shared-index count of the non-overlapping adjacent query pairs
+ * (q0,q1), (q2,q3), ... ("Adjacent-Query KV-Index Overlap in 256K DSA
+ * Training", §1; computed by batched binary search as in its §3):
+ *   out_shared[p] = | idx[2p, :len[2p]]  ∩  idx[2p+1, :len[2p+1]] |
+ * for p < S/2.  Each valid prefix must be strictly ascending (as indexer_topk
+ * writes it).  idx [S, width] int32, len [S] int32, out_shared [S/2] int32. */
+indexer_status indexer_pair_overlap(const int32_t* idx, const int32_t* len,
+                                    int64_t S, int32_t width,
+                                    int32_t* out_shared, void* stream);
+
+/* Synchronises `stream`, then reads the device status word that indexer_topk
+ * keeps in `workspace` (0 = no fault).  Bit 0: a pipeline wait in the kernel
+ * gave up after its time limit (the result is not valid); bit 1: a candidate
+ * buffer would have overflowed (never expected; the result is not valid).
+ * Also clears the word.  Host pointer `flags`. */
+indexer_status indexer_read_status(void* workspace, int32_t* flags, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* indexer_status_string(indexer_status s);
+
+/* Version of this ABI (incremented on incompatible change). */
+int32_t indexer_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HWR_INDEXER_H */
