@@ -207,7 +207,9 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
 
   CUtensorMap tm_q, tm_k;
   if (!encode_2d(&tm_q, q, fp8, p->S * p->H, p->D, pl.var.q_box_rows)) return INDEXER_ECUDA;
-  if (!encode_2d(&tm_k, keys, fp8, pl.n_keys, p->D, 128)) return INDEXER_ECUDA;
+  // With no complete pool (a sequence shorter than one pool) no key tile is
+  // ever loaded; the map still needs a non-empty extent.
+  if (!encode_2d(&tm_k, keys, fp8, pl.n_keys > 0 ? pl.n_keys : 1, p->D, 128)) return INDEXER_ECUDA;
 
   ScoreParams sp;
   sp.S = p->S;

@@ -103,7 +103,7 @@ def assert_tolerant(wl, gpu, ref, rows, rel=REL, min_recall=0.9999):
             near = np.abs(s_ref - tau) <= rel * abs(tau)
             assert near.all(), ("index sets differ away from the threshold", t, keys[~near][:8],
                                 s_ref[~near][:8], tau)
-        recalls.append(len(sa & sb) / max(len(sb), 1))
+        recalls.append(len(sa & sb) / len(sb) if sb else float(not sa))
         # scores of the selected keys
         sel = gs[r, : L - ((g + 1) % m if m > 1 else 0)].astype(np.float64)
         if sel.size:
