@@ -10,6 +10,7 @@ Workloads (names carry their sizes):
                     [-3, 3] and w in {-2..2}: every score is an exact integer.
   dsa_prefill_64k   S=T=65,536, H=64, D=128, K=2,048, token causal, N(0,1)
                     bf16 q, k; w ~ N(0, 1/H) fp32 (DSA prefill).
+  dsa_prefill_16k   the same at S=T=16,384 (a profiling-sized case).
   csa_m4_256k       S=262,144 queries over T=65,536 compressed keys (m=4),
                     H=64, D=128, K=2,048 (V4-Flash-like CSA indexer shape).
   pooled_tail_128k  S=T=131,072 tokens, pools of 4 (32,768 pools), H=32,
@@ -60,6 +61,8 @@ WORKLOADS = {
                              seed=0, values="int"),
     "dsa_prefill_64k": Workload("dsa_prefill_64k", S=65536, T=65536, H=64,
                                 D=128, K=2048, seed=1),
+    "dsa_prefill_16k": Workload("dsa_prefill_16k", S=16384, T=16384, H=64,
+                                D=128, K=2048, seed=5),
     "csa_m4_256k": Workload("csa_m4_256k", S=262144, T=65536, H=64, D=128,
                             K=2048, visibility=COMPRESSED, ratio=4, seed=2),
     "pooled_tail_128k": Workload("pooled_tail_128k", S=131072, T=131072, H=32,
