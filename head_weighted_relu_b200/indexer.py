@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
                 3: "INDEXER_EUNSUPPORTED", 4: "INDEXER_ECUDA", 5: "INDEXER_EDEVICE"}
 
 # every symbol include/hwr_indexer.h declares
-EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_pool_keys",
+EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_topk_noalloc",
+           "indexer_pool_keys",
            "indexer_pair_overlap", "indexer_read_status", "indexer_status_string",
            "indexer_abi_version")
 
@@ -57,6 +58,7 @@ def _load():
     lib.indexer_out_width.argtypes = [P, ctypes.POINTER(i32)]
     lib.indexer_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
     lib.indexer_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.indexer_pool_keys.argtypes = [vp, i64, i32, vp, i32, vp, vp]
     lib.indexer_pair_overlap.argtypes = [vp, vp, i64, i32, vp, vp]
     lib.indexer_read_status.argtypes = [vp, ctypes.POINTER(i32), vp]
@@ -113,6 +115,17 @@ def indexer_topk(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len
         ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
         _ptr(pool_coef), _ptr(out_idx), _ptr(out_len), _ptr(out_score), _ptr(workspace),
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def indexer_topk_noalloc(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len,
+                         out_score, stream=None):
+    """indexer_topk without a workspace: for callers that cannot allocate device
+    memory.  Scratch is the library's fixed 64 MiB device array; larger problems
+    raise IndexerError (INDEXER_EWORKSPACE).  Calls share that array, so calls
+    that could overlap on the GPU must be serialised."""
+    _check("indexer_topk_noalloc", _lib.indexer_topk_noalloc(
+        ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
+        _ptr(pool_coef), _ptr(out_idx), _ptr(out_len), _ptr(out_score), _stream(stream)))
 
 
 def indexer_pool_keys(k, T_tokens, D, pool_coef, ratio, out_kp, stream=None):

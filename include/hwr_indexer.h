@@ -121,6 +121,33 @@ indexer_status indexer_topk(const indexer_problem* p,
                             void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* indexer_topk for callers that cannot allocate device memory.  This entry
+ * point has no counterpart in the source pages; it exists for code that must
+ * not call cudaMalloc or any other allocator where it runs the indexer -- for
+ * example inside an allocator or memory-pool hook, in a plugin whose host
+ * framework owns every device allocation, or in a program that forbids
+ * allocation after start-up.
+ *   Same arguments and result as indexer_topk, minus the workspace: scratch
+ *   comes from one fixed 64 MiB array in the library's device image, which
+ *   every GPU that loads the library holds until the process exits.
+ *   Problems whose indexer_workspace_bytes exceeds 64 MiB are rejected with
+ *   INDEXER_EWORKSPACE before anything is launched (on a 148-SM B200 with
+ *   H = 64 that allows budgets up to K = 3,456).
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Nothing here allocates.  All calls share the one array and it keeps the
+ *   previous call's contents (each call clears what must start at zero), so
+ *   calls that may overlap on the GPU -- on different streams, or from
+ *   different host threads -- race and corrupt each other's results;
+ *   serialise them.  indexer_read_status does not apply to this entry point
+ *   (there is no workspace to pass it). */
+indexer_status indexer_topk_noalloc(const indexer_problem* p,
+                                    const void* q, const void* k, const float* w,
+                                    const float* q_scale, const float* k_scale,
+                                    const void* pool_coef,
+                                    int32_t* out_idx, int32_t* out_len, float* out_score,
+                                    void* stream);
+
 /* Pool formation alone (the first step of POOLED):
  *   kp[p, d] = RNE_bf16( exact sum_{j<ratio} c[j, d] * k[ratio*p + j, d] )
  * for p < T_tokens / ratio; k [T_tokens, D] bf16, pool_coef [ratio, D] bf16,
