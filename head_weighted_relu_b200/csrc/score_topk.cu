@@ -53,6 +53,7 @@ struct WgState {
   int32_t wc[NQA][4];    // per-warp pass counts of the current tile
   uint32_t red[16];      // reduction scratch
   int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
+  int32_t ccnt[33 * 4];  // per-(register slot, warp) kept counts of a register-resident compaction
 };
 
 template <int STAGES>
@@ -127,16 +128,19 @@ template <int H, int QPC>
 __device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float* w, float* s) {
 #pragma unroll
   for (int qq = 0; qq < QPC; ++qq) {
-    float a0 = 0.f, a1 = 0.f;
+    // two interleaved partial sums (even / odd heads) in one packed FMA
+    float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
     for (int h = 0; h < H; h += 4) {
       const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
-      a0 = fmaf(wv.x, fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f), a0);
-      a1 = fmaf(wv.y, fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f), a1);
-      a0 = fmaf(wv.z, fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f), a0);
-      a1 = fmaf(wv.w, fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f), a1);
+      const float2 r01 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f),
+                                     fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f));
+      const float2 r23 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f),
+                                     fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f));
+      acc = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc);
+      acc = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc);
     }
-    s[qq] = a0 + a1;
+    s[qq] = acc.x + acc.y;
   }
 }
 
@@ -285,6 +289,223 @@ __device__ int wg_compact(const uint2* buf, int n, Cut c, bool keep_all, int32_t
     if (keep) emit(running + prior + __popc(bal & ((1u << lane) - 1u)), e);
     running += tot;
     par ^= 1;
+  }
+  named_bar(bar_id, kBM);
+  return running;
+}
+
+// ------------------------------------------------------------------------
+// Register-resident selection: the warpgroup holds the whole candidate
+// buffer in registers (entry r*128 + etid in thread etid's slot r), so every
+// pass over it runs without memory round trips.  Used whenever the buffer
+// fits (capacity <= 4,224 entries, i.e. budgets up to 2,048).
+// ------------------------------------------------------------------------
+constexpr int kRegEntries = 33;
+constexpr int kRegCap = kRegEntries * kBM;
+
+struct RegBuf {
+  uint32_t key[kRegEntries];
+  uint32_t idx[kRegEntries];
+};
+
+__device__ __forceinline__ void rb_load(RegBuf& b, const uint2* buf, int n, int etid) {
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r) {
+    const int i = r * kBM + etid;
+    uint2 e = make_uint2(0u, 0u);
+    if (i < n) e = buf[i];
+    b.key[r] = e.x;
+    b.idx[r] = e.y;
+  }
+}
+
+// The value ranked: the ordered score, or ~index (so that larger = lower index).
+__device__ __forceinline__ uint32_t rb_field(const RegBuf& b, int r, bool idx_field) {
+  return idx_field ? ~b.idx[r] : b.key[r];
+}
+
+// Largest and smallest ranked value over the valid entries (only those whose
+// ordered score equals fval when `filt`).  The next pass's barriers order the
+// reuse of `red`.
+__device__ void rb_maxmin(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t& mx,
+                          uint32_t& mn, uint32_t* red, int etid, int bar_id) {
+  const int lane = etid & 31, wq = etid >> 5;
+  mx = 0u;
+  mn = 0xFFFFFFFFu;
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r) {
+    if (r * kBM + etid < n && (!filt || b.key[r] == fval)) {
+      const uint32_t f = rb_field(b, r, idx_field);
+      mx = max(mx, f);
+      mn = min(mn, f);
+    }
+  }
+  mx = warp_max_u32(mx);
+  mn = warp_min_u32(mn);
+  if (lane == 0) {
+    red[wq] = mx;
+    red[4 + wq] = mn;
+  }
+  named_bar(bar_id, kBM);
+  mx = max(max(red[0], red[1]), max(red[2], red[3]));
+  mn = min(min(red[4], red[5]), min(red[6], red[7]));
+}
+
+struct Digit {
+  uint32_t d;      // the digit holding the rank-th largest
+  uint32_t above;  // entries in higher digits (this pass)
+  uint32_t cnt;    // entries in digit d
+};
+
+// One MSB-first radix pass over bits [lo - width, lo) of the valid entries
+// whose bits [lo, 32) equal prefix's.  Bin b of the histogram sits at word
+// ((b % per) << 7) + b / per, so the 128 owner threads, each summing `per`
+// consecutive bins, read distinct banks.
+__device__ Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t prefix, int lo,
+                         int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
+  const int lane = etid & 31, wq = etid >> 5;
+  const int shift = lo - width;
+  const int nb = 1 << width;
+  const int lper = width > 7 ? width - 7 : 0;
+  const int per = 1 << lper;
+  for (int i = etid; i < nb; i += kBM) hist[i] = 0u;
+  named_bar(bar_id, kBM);
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r) {
+    if (r * kBM + etid < n && (!filt || b.key[r] == fval)) {
+      const uint32_t f = rb_field(b, r, idx_field);
+      if (lo >= 32 || (f >> lo) == (prefix >> lo)) {
+        const uint32_t bin = (f >> shift) & static_cast<uint32_t>(nb - 1);
+        atomicAdd(&hist[((bin & static_cast<uint32_t>(per - 1)) << 7) + (bin >> lper)], 1u);
+      }
+    }
+  }
+  named_bar(bar_id, kBM);
+  const bool owner = etid < (nb >> lper);
+  uint32_t local = 0u;
+  if (owner)
+    for (int k = 0; k < per; ++k) local += hist[(k << 7) + etid];
+  uint32_t incl = local;  // sum over lanes >= this lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_down_sync(kFullMask, incl, o);
+    if (lane + o < 32) incl += t;
+  }
+  if (lane == 0) red[wq] = incl;
+  named_bar(bar_id, kBM);
+  uint32_t higher = 0u;
+  for (int w2 = wq + 1; w2 < 4; ++w2) higher += red[w2];
+  const uint32_t excl = incl - local + higher;  // entries in bins owned by higher threads
+  if (owner && local > 0u && excl < rank && rank <= excl + local) {
+    uint32_t acc = excl;
+    for (int k = per - 1; k >= 0; --k) {
+      const uint32_t h = hist[(k << 7) + etid];
+      if (acc + h >= rank) {
+        red[8] = static_cast<uint32_t>(etid * per + k);
+        red[9] = acc;
+        red[10] = h;
+        break;
+      }
+      acc += h;
+    }
+  }
+  named_bar(bar_id, kBM);
+  const Digit out{red[8], red[9], red[10]};
+  named_bar(bar_id, kBM);
+  return out;
+}
+
+// A cut of a buffer to its top `ksel`: keep key >= v when `ge`, otherwise keep
+// key > v, or key == v and index <= icut.  `kept` = entries the cut keeps.
+struct RegCut {
+  uint32_t v;
+  uint32_t icut;
+  bool ge;
+  int kept;
+};
+
+// MSB-first radix select of the ksel-th largest (ordered score, then lowest
+// index), starting below the bits every entry shares.  With `approx`, stops
+// after the first pass if keeping the whole digit that holds the ksel-th entry
+// keeps at most `room` entries: a safe lower bound for a running threshold.
+__device__ RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int room, uint32_t* hist,
+                         uint32_t* red, int etid, int bar_id) {
+  uint32_t mx, mn;
+  rb_maxmin(b, n, false, false, 0u, mx, mn, red, etid, bar_id);
+  uint32_t prefix = mx, above = 0u, cnt = static_cast<uint32_t>(n), rank = ksel;
+  if (mx != mn) {
+    int lo = 32 - __clz(mx ^ mn);
+    prefix = lo >= 32 ? 0u : (mx >> lo) << lo;
+    bool first = true;
+    while (lo > 0) {
+      const int width = lo < 11 ? lo : 11;
+      const Digit dg = rb_pass(b, n, false, false, 0u, prefix, lo, width, rank, hist, red, etid, bar_id);
+      lo -= width;
+      prefix |= dg.d << lo;
+      above += dg.above;
+      rank -= dg.above;
+      cnt = dg.cnt;
+      if (approx && first && static_cast<int>(above + cnt) <= room)
+        return {prefix, 0u, true, static_cast<int>(above + cnt)};
+      first = false;
+    }
+  }
+  // prefix is now v, the ksel-th largest ordered score; `rank` of the `cnt`
+  // entries tied at v make the cut
+  if (rank >= cnt) return {prefix, 0xFFFFFFFFu, false, static_cast<int>(above + cnt)};
+  uint32_t imx, imn;
+  rb_maxmin(b, n, true, true, prefix, imx, imn, red, etid, bar_id);
+  uint32_t ip = imx;
+  if (imx != imn) {
+    int lo = 32 - __clz(imx ^ imn);
+    ip = lo >= 32 ? 0u : (imx >> lo) << lo;
+    uint32_t irank = rank;
+    while (lo > 0) {
+      const int width = lo < 11 ? lo : 11;
+      const Digit dg = rb_pass(b, n, true, true, prefix, ip, lo, width, irank, hist, red, etid, bar_id);
+      lo -= width;
+      ip |= dg.d << lo;
+      irank -= dg.above;
+    }
+  }
+  return {prefix, ~ip, false, static_cast<int>(ksel)};
+}
+
+// Calls emit(pos, key, idx) for every kept entry in buffer (key) order;
+// returns the number kept.  All reads are from registers, so emitting back
+// into the same buffer is safe.
+template <class Emit>
+__device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all, int32_t* ccnt, int etid,
+                          int bar_id, Emit emit) {
+  const int lane = etid & 31, wq = etid >> 5;
+  auto keep_of = [&](int r) -> bool {
+    if (r * kBM + etid >= n) return false;
+    if (keep_all) return true;
+    const uint32_t k = b.key[r];
+    return c.ge ? (k >= c.v) : (k > c.v || (k == c.v && b.idx[r] <= c.icut));
+  };
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r) {
+    const uint32_t bal = __ballot_sync(kFullMask, keep_of(r));
+    if (lane == 0) ccnt[r * 4 + wq] = __popc(bal);
+  }
+  named_bar(bar_id, kBM);
+  int running = 0;
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r) {
+    if (r * kBM < n) {
+      const bool kp = keep_of(r);
+      const uint32_t bal = __ballot_sync(kFullMask, kp);
+      int prior = 0, tot = 0;
+#pragma unroll
+      for (int w2 = 0; w2 < 4; ++w2) {
+        const int cc = ccnt[r * 4 + w2];
+        tot += cc;
+        prior += (w2 < wq) ? cc : 0;
+      }
+      if (kp) emit(running + prior + __popc(bal & ((1u << lane) - 1u)), b.key[r], b.idx[r]);
+      running += tot;
+    }
   }
   named_bar(bar_id, kBM);
   return running;
@@ -549,18 +770,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_bar(bar_id, kBM);
         par = np;
-        // cut buffers that could not take another full tile back to their top-K
+        // cut buffers that could not take another full tile back toward their top-K
 #pragma unroll 1
         for (int qi = 0; qi < NQA; ++qi) {
           const int n = st->cnt[par][qi];
           if (n > p.cap - kBM) {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
-            const Cut cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
-            wg_compact(buf, n, cut, false, &st->cwc[0][0], etid, bar_id,
-                       [&](int pos, uint2 e) { buf[pos] = e; });
+            int kept;
+            uint32_t thr;
+            if (n <= kRegCap) {
+              RegBuf rb;
+              rb_load(rb, buf, n, etid);
+              const RegCut c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), true, p.cap - 2 * kBM, hist,
+                                      st->red, etid, bar_id);
+              kept = rb_compact(rb, n, c, false, st->ccnt, etid, bar_id,
+                                [&](int pos, uint32_t k, uint32_t ix) { buf[pos] = make_uint2(k, ix); });
+              thr = c.ge ? c.v : (c.v == 0xFFFFFFFFu ? c.v : c.v + 1u);
+            } else {
+              const Cut cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
+              kept = wg_compact(buf, n, cut, false, &st->cwc[0][0], etid, bar_id,
+                                [&](int pos, uint2 e) { buf[pos] = e; });
+              thr = cut.v == 0xFFFFFFFFu ? cut.v : cut.v + 1u;
+            }
             if (etid == 0) {
-              st->cnt[par][qi] = p.ksel;
-              st->thr[qi] = cut.v == 0xFFFFFFFFu ? cut.v : cut.v + 1u;
+              st->cnt[par][qi] = kept;
+              st->thr[qi] = thr;
             }
             named_bar(bar_id, kBM);
           }
@@ -576,23 +810,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = st->cnt[par][qi];
         uint2* buf = cand + qi * static_cast<size_t>(p.cap);
         const bool all = n <= p.ksel;
-        Cut cut{0u, 0xFFFFFFFFu};
-        if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
         int32_t* orow = p.out_idx + t * p.width;
         float* srow = p.out_score ? p.out_score + t * p.width : nullptr;
         const int m = p.out_ratio;
-        const int kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id, [&](int pos, uint2 e) {
-          const float sc = key_to_float(e.x);
+        auto emit = [&](int pos, uint32_t k, uint32_t ix) {
+          const float sc = key_to_float(k);
           if (m == 1) {
-            orow[pos] = static_cast<int32_t>(e.y);
+            orow[pos] = static_cast<int32_t>(ix);
             if (srow) srow[pos] = sc;
           } else {
             for (int rr = 0; rr < m; ++rr) {
-              orow[pos * m + rr] = static_cast<int32_t>(e.y) * m + rr;
+              orow[pos * m + rr] = static_cast<int32_t>(ix) * m + rr;
               if (srow) srow[pos * m + rr] = sc;
             }
           }
-        });
+        };
+        int kept;
+        if (n <= kRegCap) {
+          RegBuf rb;
+          rb_load(rb, buf, n, etid);
+          RegCut c{0u, 0xFFFFFFFFu, false, n};
+          if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
+          kept = rb_compact(rb, n, c, all, st->ccnt, etid, bar_id, emit);
+        } else {
+          Cut cut{0u, 0xFFFFFFFFu};
+          if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
+          kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id,
+                            [&](int pos, uint2 e) { emit(pos, e.x, e.y); });
+        }
         int len = kept * m;
         if (m > 1) {
           const int64_t g = p.q_pos0 + t;
