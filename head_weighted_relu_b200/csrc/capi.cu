@@ -105,8 +105,8 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
     const indexer_status st = device_info(&di);
     if (st != INDEXER_OK) return st;
     pl->grid = static_cast<int32_t>(nb < di.sms ? nb : di.sms);
-    pl->cand_bytes = static_cast<size_t>(pl->grid) * 2 * pl->var.queries_per_wg * static_cast<size_t>(pl->cap) *
-                     sizeof(uint2);
+    pl->cand_bytes = static_cast<size_t>(pl->grid) * pl->var.groups * pl->var.queries_per_wg *
+                     static_cast<size_t>(pl->cap) * sizeof(uint2);
   }
   pl->kp_bytes = p->visibility == INDEXER_VIS_POOLED
                      ? align256(static_cast<size_t>(pl->n_keys) * p->D * 2)

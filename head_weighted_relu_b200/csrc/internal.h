@@ -30,7 +30,7 @@ struct ScoreParams {
   int32_t* out_idx;      // [S, width]
   int32_t* out_len;      // [S]
   float* out_score;      // [S, width] or null
-  uint2* cand;           // candidate buffers: [grid][2][queries per warpgroup][cap]
+  uint2* cand;           // candidate buffers: [grid][groups][queries per group][cap]
   uint32_t* status;      // device status word
 };
 
@@ -38,7 +38,8 @@ struct ScoreParams {
 struct ScoreVariant {
   const void* fn;         // kernel function
   int queries_per_block;  // QB
-  int queries_per_wg;     // NQA
+  int queries_per_wg;     // queries owned by one epilogue warpgroup
+  int groups;             // epilogue warpgroups per CTA
   int q_box_rows;         // rows of the q TMA box
   int box_elems;          // inner extent of every TMA box (128 bytes)
   int smem_bytes;         // dynamic shared memory
@@ -50,8 +51,9 @@ bool score_variant(int H, int D, bool fp8, ScoreVariant* out);
 
 // Candidate-buffer capacity per query for a selection budget of ksel keys.
 inline int candidate_capacity(int ksel) {
-  int c = ((2 * ksel + 127) / 128) * 128 + 128;
-  return c;
+  // room for the budget, plus at least as much again for new candidates
+  int c = ((2 * ksel + 127) / 128) * 128;
+  return c < ksel + 256 ? ((ksel + 256 + 127) / 128) * 128 : c;
 }
 
 cudaError_t launch_pool_keys(const void* k, int64_t n_pools, int D, const void* coef, int ratio, void* out,

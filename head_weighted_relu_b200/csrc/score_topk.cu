@@ -11,15 +11,16 @@
 // partition-merge top-K instead of materialising scores; this kernel streams
 // keys in ascending order and merges into a running selection.
 //
-// One persistent CTA per SM, 10 warps:
+// One persistent CTA per SM, 20 warps:
 //   warp 0      TMA producer: the query block's q rows once, then key tiles of
 //               128 rows through a ring of shared-memory stages;
 //   warp 1      MMA issuer: for each key tile, two accumulators
 //               acc[a][key, (query, head)] = k_tile . q_block[a]^T
 //               (M = 128 keys = TMEM lanes, N = queries x heads <= 256 columns,
 //               K = D), tcgen05.mma with FP32 accumulation in TMEM;
-//   warps 2..9  two epilogue warpgroups, one per accumulator.  Each thread owns
-//               one key (one TMEM lane) and, for every query of its group,
+//   warps 4..19 four epilogue warpgroups, two per accumulator, each taking
+//               half of its queries.  Each thread owns one key (one TMEM
+//               lane) and, for every query of its group,
 //               reduces sum_h w[t,h] * max(acc, 0) in registers, applies the
 //               visibility mask, and appends (ordered score, key) pairs that
 //               beat the query's running threshold to a per-query candidate
@@ -39,21 +40,29 @@
 
 namespace hwr {
 
-constexpr int kThreads = 320;
+// 20 warps: warpgroup 0 = TMA producer, MMA issuer and two idle warps;
+// warpgroups 1..4 = epilogue.  Registers at launch: 640 x 96 = 61,440.
+// Warpgroup 0 drops to 32 per thread and the epilogue takes 112:
+// 128 x 32 + 512 x 112 = 61,440 (per SMSP: 32*32 + 4*112*32 = 15,360 <= 16,384).
+constexpr int kThreads = 640;
+constexpr int kRegsControl = 32;
+constexpr int kRegsEpilogue = 112;
+constexpr int kEpiGroups = 4;
 constexpr int kBM = 128;                         // keys per tile = MMA M = TMEM lanes
-constexpr int kHistBins = 2048;                  // 11-bit radix digits
+constexpr int kDigitBits = 10;                   // radix digit width
+constexpr int kHistBins = 1 << kDigitBits;
 constexpr int kSmemLimit = 232448;               // 227 KB opt-in shared memory per CTA
 constexpr uint64_t kWaitLimitNs = 4000000000ull; // give up a pipeline wait after 4 s
 
-template <int NQA>
+template <int NQ>
 struct WgState {
-  uint32_t thr[NQA];     // a candidate is appended iff its ordered score >= thr
-  int32_t cnt[2][NQA];   // candidates held, double-buffered by tile parity
-  int32_t nvis[NQA];     // keys visible to each query of the group
-  int32_t wc[NQA][4];    // per-warp pass counts of the current tile
+  uint32_t thr[NQ];      // a candidate is appended iff its ordered score >= thr
+  int32_t cnt[2][NQ];    // candidates held, double-buffered by tile parity
+  int32_t nvis[NQ];      // keys visible to each query of the group
+  int32_t wc[2][NQ][4];  // per-warp pass counts, double-buffered by tile parity
   uint32_t red[16];      // reduction scratch
   int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
-  int32_t ccnt[33 * 4];  // per-(register slot, warp) kept counts of a register-resident compaction
+  int32_t scan[4];       // per-warp totals of a register-resident compaction
 };
 
 template <int STAGES>
@@ -74,30 +83,32 @@ struct Cfg {
   static constexpr int NBOX = ROW_BYTES / 128;          // 128-byte swizzle boxes per row
   static constexpr int BOX_ELEMS = 128 / ELEM;
   static constexpr int KSTEPS = ROW_BYTES / 32;          // MMA K steps of 32 bytes
-  static constexpr int NQA = (256 / H) < 16 ? (256 / H) : 16;  // queries per accumulator
+  static constexpr int NQA = (256 / H) < 32 ? (256 / H) : 32;  // queries per accumulator
+  static constexpr int NQW = NQA / 2;                    // queries per epilogue warpgroup
   static constexpr int BN = NQA * H;                     // accumulator columns = MMA N
   static constexpr int QB = 2 * NQA;                     // queries per block
-  static constexpr int CHUNKS = BN / 64;                 // 64-column TMEM loads per accumulator
+  static constexpr int CHUNKS_W = (BN / 2) / 64;         // 64-column TMEM loads per warpgroup
   static constexpr int QPC = 64 / H;                     // queries per 64-column load
   static constexpr int Q_ACC_BYTES = BN * ROW_BYTES;
   static constexpr int Q_BYTES = 2 * Q_ACC_BYTES;
   static constexpr int K_STAGE_BYTES = kBM * ROW_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMALL_BYTES = kHistBins * 4 * 2 + 2 * BN * 4 + 2 * (int)sizeof(WgState<NQA>);
+  static constexpr int SMALL_BYTES =
+      kHistBins * 4 * kEpiGroups + 2 * BN * 4 + kEpiGroups * (int)sizeof(WgState<NQW>);
   static constexpr int AVAIL = kSmemLimit - 1024 - Q_BYTES - SMALL_BYTES - (int)sizeof(Barriers<8>);
   static constexpr int STAGES_RAW = AVAIL / K_STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_HIST = OFF_K + STAGES * K_STAGE_BYTES;
-  static constexpr int OFF_W = OFF_HIST + kHistBins * 4 * 2;
+  static constexpr int OFF_W = OFF_HIST + kHistBins * 4 * kEpiGroups;
   static constexpr int OFF_ST = OFF_W + 2 * BN * 4;
-  static constexpr int OFF_BAR = OFF_ST + 2 * (int)sizeof(WgState<NQA>);
+  static constexpr int OFF_BAR = OFF_ST + kEpiGroups * (int)sizeof(WgState<NQW>);
   static constexpr int SMEM_BYTES = 1024 + OFF_BAR + (int)sizeof(Barriers<STAGES>);
   static constexpr uint32_t IDESC = FP8 ? idesc_e4m3<kBM, BN>() : idesc_bf16<kBM, BN>();
   static_assert(H % 4 == 0 && H <= 64, "heads");
   static_assert(ROW_BYTES % 128 == 0, "row must be whole 128-byte swizzle rows");
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "accumulator width");
+  static_assert(BN % 128 == 0 && BN >= 128 && BN <= 256, "accumulator width");
   static_assert(STAGES >= 2, "shared memory too small for a 2-stage key ring");
   static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
   static_assert(OFF_K % 1024 == 0 && K_STAGE_BYTES % 1024 == 0 && Q_ACC_BYTES % 1024 == 0, "swizzle alignment");
@@ -128,8 +139,10 @@ template <int H, int QPC>
 __device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float* w, float* s) {
 #pragma unroll
   for (int qq = 0; qq < QPC; ++qq) {
-    // two interleaved partial sums (even / odd heads) in one packed FMA
-    float2 acc = make_float2(0.f, 0.f);
+    // four independent packed partial sums (heads h mod 8 in pairs) keep the
+    // FMA dependency chains short
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                     make_float2(0.f, 0.f)};
 #pragma unroll
     for (int h = 0; h < H; h += 4) {
       const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
@@ -137,10 +150,11 @@ __device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float
                                      fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f));
       const float2 r23 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f),
                                      fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f));
-      acc = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc);
-      acc = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc);
+      const int c = (h >> 2) & 1;
+      acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
+      acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
     }
-    s[qq] = acc.x + acc.y;
+    s[qq] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
   }
 }
 
@@ -186,7 +200,7 @@ __device__ SelResult wg_radix_select(const uint2* buf, int n, uint32_t rank, boo
   uint32_t prefix = lo >= 32 ? 0u : (mx >> lo) << lo;
   uint32_t rem = rank, above = 0u, eq = 0u;
   while (lo > 0) {
-    const int width = lo < 11 ? lo : 11;
+    const int width = lo < kDigitBits ? lo : kDigitBits;
     const int shift = lo - width;
     const int nb = 1 << width;
     for (int i = etid; i < nb; i += kBM) hist[i] = 0u;
@@ -296,11 +310,12 @@ __device__ int wg_compact(const uint2* buf, int n, Cut c, bool keep_all, int32_t
 
 // ------------------------------------------------------------------------
 // Register-resident selection: the warpgroup holds the whole candidate
-// buffer in registers (entry r*128 + etid in thread etid's slot r), so every
-// pass over it runs without memory round trips.  Used whenever the buffer
-// fits (capacity <= 4,224 entries, i.e. budgets up to 2,048).
+// buffer in registers, thread etid holding the contiguous entries
+// [32*etid, 32*etid + 32), so every pass over it runs without memory round
+// trips and order-preserving compaction needs one prefix scan.  Used whenever
+// the buffer fits (capacity <= 4,096 entries, i.e. budgets up to 2,048).
 // ------------------------------------------------------------------------
-constexpr int kRegEntries = 33;
+constexpr int kRegEntries = 32;
 constexpr int kRegCap = kRegEntries * kBM;
 
 struct RegBuf {
@@ -309,13 +324,16 @@ struct RegBuf {
 };
 
 __device__ __forceinline__ void rb_load(RegBuf& b, const uint2* buf, int n, int etid) {
+  const int base = etid * kRegEntries;
+  const uint4* v = reinterpret_cast<const uint4*>(buf + base);
 #pragma unroll
-  for (int r = 0; r < kRegEntries; ++r) {
-    const int i = r * kBM + etid;
-    uint2 e = make_uint2(0u, 0u);
-    if (i < n) e = buf[i];
+  for (int r = 0; r < kRegEntries; r += 2) {
+    uint4 e = make_uint4(0u, 0u, 0u, 0u);
+    if (base + r < n) e = v[r >> 1];  // n entries are valid; the pair's tail is masked below
     b.key[r] = e.x;
     b.idx[r] = e.y;
+    b.key[r + 1] = e.z;
+    b.idx[r + 1] = e.w;
   }
 }
 
@@ -330,11 +348,12 @@ __device__ __forceinline__ uint32_t rb_field(const RegBuf& b, int r, bool idx_fi
 __device__ void rb_maxmin(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t& mx,
                           uint32_t& mn, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
+  const int base = etid * kRegEntries;
   mx = 0u;
   mn = 0xFFFFFFFFu;
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r) {
-    if (r * kBM + etid < n && (!filt || b.key[r] == fval)) {
+    if (base + r < n && (!filt || b.key[r] == fval)) {
       const uint32_t f = rb_field(b, r, idx_field);
       mx = max(mx, f);
       mn = min(mn, f);
@@ -364,6 +383,7 @@ struct Digit {
 __device__ Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t prefix, int lo,
                          int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
+  const int base = etid * kRegEntries;
   const int shift = lo - width;
   const int nb = 1 << width;
   const int lper = width > 7 ? width - 7 : 0;
@@ -372,7 +392,7 @@ __device__ Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint
   named_bar(bar_id, kBM);
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r) {
-    if (r * kBM + etid < n && (!filt || b.key[r] == fval)) {
+    if (base + r < n && (!filt || b.key[r] == fval)) {
       const uint32_t f = rb_field(b, r, idx_field);
       if (lo >= 32 || (f >> lo) == (prefix >> lo)) {
         const uint32_t bin = (f >> shift) & static_cast<uint32_t>(nb - 1);
@@ -438,7 +458,7 @@ __device__ RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int
     prefix = lo >= 32 ? 0u : (mx >> lo) << lo;
     bool first = true;
     while (lo > 0) {
-      const int width = lo < 11 ? lo : 11;
+      const int width = lo < kDigitBits ? lo : kDigitBits;
       const Digit dg = rb_pass(b, n, false, false, 0u, prefix, lo, width, rank, hist, red, etid, bar_id);
       lo -= width;
       prefix |= dg.d << lo;
@@ -461,7 +481,7 @@ __device__ RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int
     ip = lo >= 32 ? 0u : (imx >> lo) << lo;
     uint32_t irank = rank;
     while (lo > 0) {
-      const int width = lo < 11 ? lo : 11;
+      const int width = lo < kDigitBits ? lo : kDigitBits;
       const Digit dg = rb_pass(b, n, true, true, prefix, ip, lo, width, irank, hist, red, etid, bar_id);
       lo -= width;
       ip |= dg.d << lo;
@@ -471,44 +491,44 @@ __device__ RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int
   return {prefix, ~ip, false, static_cast<int>(ksel)};
 }
 
-// Calls emit(pos, key, idx) for every kept entry in buffer (key) order;
-// returns the number kept.  All reads are from registers, so emitting back
-// into the same buffer is safe.
+// Calls emit(pos, key, idx) for every kept entry, pos counting kept entries in
+// buffer (key) order; returns the number kept.  Each thread counts its kept
+// entries, one scan over the warpgroup gives its first position.  All reads
+// are from registers, so emitting back into the same buffer is safe.
 template <class Emit>
-__device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all, int32_t* ccnt, int etid,
+__device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all, int32_t* red_i, int etid,
                           int bar_id, Emit emit) {
   const int lane = etid & 31, wq = etid >> 5;
+  const int base = etid * kRegEntries;
   auto keep_of = [&](int r) -> bool {
-    if (r * kBM + etid >= n) return false;
+    if (base + r >= n) return false;
     if (keep_all) return true;
     const uint32_t k = b.key[r];
     return c.ge ? (k >= c.v) : (k > c.v || (k == c.v && b.idx[r] <= c.icut));
   };
+  int mine = 0;
 #pragma unroll
-  for (int r = 0; r < kRegEntries; ++r) {
-    const uint32_t bal = __ballot_sync(kFullMask, keep_of(r));
-    if (lane == 0) ccnt[r * 4 + wq] = __popc(bal);
+  for (int r = 0; r < kRegEntries; ++r) mine += keep_of(r) ? 1 : 0;
+  int incl = mine;  // inclusive prefix over lanes <= this lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(kFullMask, incl, o);
+    if (lane >= o) incl += t;
   }
+  if (lane == 31) red_i[wq] = incl;
   named_bar(bar_id, kBM);
-  int running = 0;
+  int pos = incl - mine, total = 0;
 #pragma unroll
-  for (int r = 0; r < kRegEntries; ++r) {
-    if (r * kBM < n) {
-      const bool kp = keep_of(r);
-      const uint32_t bal = __ballot_sync(kFullMask, kp);
-      int prior = 0, tot = 0;
-#pragma unroll
-      for (int w2 = 0; w2 < 4; ++w2) {
-        const int cc = ccnt[r * 4 + w2];
-        tot += cc;
-        prior += (w2 < wq) ? cc : 0;
-      }
-      if (kp) emit(running + prior + __popc(bal & ((1u << lane) - 1u)), b.key[r], b.idx[r]);
-      running += tot;
-    }
+  for (int w2 = 0; w2 < 4; ++w2) {
+    const int t = red_i[w2];
+    total += t;
+    pos += (w2 < wq) ? t : 0;
   }
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r)
+    if (keep_of(r)) emit(pos++, b.key[r], b.idx[r]);
   named_bar(bar_id, kBM);
-  return running;
+  return total;
 }
 
 // ------------------------------------------------------------------------
@@ -520,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const ScoreParams p) {
   using C = Cfg<H, D, FP8>;
   constexpr int NQA = C::NQA;
+  constexpr int NQW = C::NQW;
   constexpr int BN = C::BN;
   constexpr int QB = C::QB;
   constexpr int STAGES = C::STAGES;
@@ -528,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* hist_base = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
   float* wsm_base = reinterpret_cast<float*>(smem + C::OFF_W);
-  WgState<NQA>* states = reinterpret_cast<WgState<NQA>*>(smem + C::OFF_ST);
+  WgState<NQW>* states = reinterpret_cast<WgState<NQW>*>(smem + C::OFF_ST);
   Barriers<STAGES>* bars = reinterpret_cast<Barriers<STAGES>*>(smem + C::OFF_BAR);
 
   const int warp = threadIdx.x >> 5;
@@ -543,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->qempty, 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->accfull[a], 1);
-      mbar_init(&bars->accempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&bars->accempty[a], 8);  // one arrival per warp of the two groups sharing it
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -559,6 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = bars->tmem_slot;
   volatile int* abort_flag = &bars->abort;
 
+  // The two register classes never rejoin: each branch ends in the same named
+  // barrier (id 15, all threads), after which warp 1 frees TMEM.
+  constexpr int kExitBar = 15;
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -662,16 +688,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0u, abort_flag, kWaitLimitNs);
     }
+  }
+  __syncwarp();  // lane 0 of warps 0 and 1 rejoins its warp before the aligned barrier
+  tc_fence_before();
+  named_bar(kExitBar, kThreads);
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
   } else {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpilogue));
+  {
     // ------------------------------------------------------ epilogue warpgroups
-    const int wg = (warp - 2) >> 2;
+    const int eg = (warp - 4) >> 2;    // epilogue group 0..3
+    const int acc = eg >> 1;           // the accumulator it drains
+    const int half = eg & 1;           // which half of that accumulator's queries
     const int wq = warp & 3;           // TMEM lane quarter accessible to this warp
     const int etid = wq * 32 + lane;   // key row within the tile == order within the group
-    const int bar_id = 1 + wg;
-    WgState<NQA>* st = states + wg;
-    float* wsm = wsm_base + wg * BN;
-    uint32_t* hist = hist_base + wg * kHistBins;
-    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(wg * BN);
+    const int bar_id = 1 + eg;
+    WgState<NQW>* st = states + eg;
+    float* wsm = wsm_base + eg * (BN / 2);
+    uint32_t* hist = hist_base + eg * kHistBins;
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) +
+                           static_cast<uint32_t>(acc * BN + half * (BN / 2));
     uint32_t af_ph = 0u;
     int par = 0;
     bool failed = false;
@@ -679,11 +716,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
       if (b < 0) break;
       const int nt = tiles_of_block<QB>(p, b);
-      const int64_t tq0 = static_cast<int64_t>(b) * QB + wg * NQA;
-      uint2* cand = p.cand + (static_cast<size_t>(blockIdx.x) * 2 + wg) * NQA * static_cast<size_t>(p.cap);
+      const int64_t tq0 = static_cast<int64_t>(b) * QB + acc * NQA + half * NQW;
+      uint2* cand = p.cand + (static_cast<size_t>(blockIdx.x) * kEpiGroups + eg) * NQW * static_cast<size_t>(p.cap);
 
       named_bar(bar_id, kBM);  // the previous block is completely done with the state
-      for (int i = etid; i < BN; i += kBM) {
+      for (int i = etid; i < BN / 2; i += kBM) {
         const int64_t t = tq0 + i / H;
         float v = 0.f;
         if (t < p.S) {
@@ -692,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         wsm[i] = v;
       }
-      if (etid < NQA) {
+      if (etid < NQW) {
         const int64_t t = tq0 + etid;
         st->nvis[etid] = t < p.S ? n_visible(p, p.q_pos0 + t) : 0;
         st->cnt[par][etid] = 0;
@@ -702,55 +739,54 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       for (int j = 0; j < nt; ++j) {
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(&bars->accfull[wg], af_ph, abort_flag, kWaitLimitNs);
+        if (lane == 0) ok = mbar_wait(&bars->accfull[acc], af_ph, abort_flag, kWaitLimitNs);
         ok = __shfl_sync(kFullMask, ok ? 1 : 0, 0) != 0;
         af_ph ^= 1u;
-        float s[NQA];
+        float s[NQW];
 #pragma unroll
-        for (int qi = 0; qi < NQA; ++qi) s[qi] = 0.f;
+        for (int qi = 0; qi < NQW; ++qi) s[qi] = 0.f;
         if (ok) {
           tc_fence_after();
-          uint32_t ra[64], rb[64];
-          tmem_ld_x64(tbase, ra);
-          tmem_wait_ld(ra);
+          uint32_t ra[64];
 #pragma unroll
-          for (int c = 0; c < C::CHUNKS; ++c) {
-            if ((c & 1) == 0) {
-              if (c + 1 < C::CHUNKS) tmem_ld_x64(tbase + (c + 1) * 64, rb);
-              score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
-              if (c + 1 < C::CHUNKS) tmem_wait_ld(rb);
-            } else {
-              if (c + 1 < C::CHUNKS) tmem_ld_x64(tbase + (c + 1) * 64, ra);
-              score_chunk<H, C::QPC>(rb, wsm + c * 64, s + c * C::QPC);
-              if (c + 1 < C::CHUNKS) tmem_wait_ld(ra);
+          for (int c = 0; c < C::CHUNKS_W; ++c) {
+            tmem_ld_x64(tbase + c * 64, ra);
+            tmem_wait_ld(ra);
+            if (c + 1 == C::CHUNKS_W) {
+              // everything this warp needs from TMEM is in registers: hand the
+              // accumulator back before the last chunk's arithmetic
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->accempty[acc]);
             }
+            score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->accempty[wg]);
         }
         const int32_t key = j * kBM + etid;
         if constexpr (FP8) {
           const float ks = key < p.n_keys ? p.k_scale[key] : 0.f;
 #pragma unroll
-          for (int qi = 0; qi < NQA; ++qi) s[qi] *= ks;
+          for (int qi = 0; qi < NQW; ++qi) s[qi] *= ks;
         }
         // pass flags and per-warp counts
 #pragma unroll
-        for (int qi = 0; qi < NQA; ++qi) {
+        for (int qi = 0; qi < NQW; ++qi) {
           const uint32_t okey = ordered_key(__fadd_rn(s[qi], 0.f));
           const bool pass = ok && key < st->nvis[qi] && okey >= st->thr[qi];
           const uint32_t bal = __ballot_sync(kFullMask, pass);
-          if (lane == 0) st->wc[qi][wq] = __popc(bal);
+          if (lane == 0) st->wc[par][qi][wq] = __popc(bal);
         }
         if (named_bar_or(bar_id, kBM, !ok)) {
           failed = true;
           break;
         }
-        // ordered append: position = held + earlier warps + earlier lanes
+        // ordered append: position = held + earlier warps + earlier lanes.  No
+        // barrier follows: every thread knows the new counts, and the state read
+        // here is double-buffered by tile parity.
         const int np = par ^ 1;
+        int newcnt[NQW];
 #pragma unroll
-        for (int qi = 0; qi < NQA; ++qi) {
+        for (int qi = 0; qi < NQW; ++qi) {
           const uint32_t okey = ordered_key(__fadd_rn(s[qi], 0.f));
           const bool pass = key < st->nvis[qi] && okey >= st->thr[qi];
           const uint32_t bal = __ballot_sync(kFullMask, pass);
@@ -758,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int prior = 0, tot = 0;
 #pragma unroll
           for (int w2 = 0; w2 < 4; ++w2) {
-            const int cc = st->wc[qi][w2];
+            const int cc = st->wc[par][qi][w2];
             tot += cc;
             prior += (w2 < wq) ? cc : 0;
           }
@@ -766,14 +802,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int pos = held + prior + __popc(bal & ((1u << lane) - 1u));
             cand[qi * static_cast<size_t>(p.cap) + pos] = make_uint2(okey, static_cast<uint32_t>(key));
           }
+          newcnt[qi] = held + tot;
           if (etid == qi) st->cnt[np][qi] = held + tot;
         }
-        named_bar(bar_id, kBM);
         par = np;
         // cut buffers that could not take another full tile back toward their top-K
-#pragma unroll 1
-        for (int qi = 0; qi < NQA; ++qi) {
-          const int n = st->cnt[par][qi];
+        bool any_full = false;
+#pragma unroll
+        for (int qi = 0; qi < NQW; ++qi) any_full |= newcnt[qi] > p.cap - kBM;
+        if (any_full) named_bar(bar_id, kBM);  // every append of this tile is visible
+#pragma unroll
+        for (int qi = 0; qi < NQW; ++qi) {
+          const int n = newcnt[qi];
           if (n > p.cap - kBM) {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
             int kept;
@@ -783,7 +823,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               rb_load(rb, buf, n, etid);
               const RegCut c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), true, p.cap - 2 * kBM, hist,
                                       st->red, etid, bar_id);
-              kept = rb_compact(rb, n, c, false, st->ccnt, etid, bar_id,
+              kept = rb_compact(rb, n, c, false, st->scan, etid, bar_id,
                                 [&](int pos, uint32_t k, uint32_t ix) { buf[pos] = make_uint2(k, ix); });
               thr = c.ge ? c.v : (c.v == 0xFFFFFFFFu ? c.v : c.v + 1u);
             } else {
@@ -804,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // final selection of each query of the group, written in key order
 #pragma unroll 1
-      for (int qi = 0; qi < NQA; ++qi) {
+      for (int qi = 0; qi < NQW; ++qi) {
         const int64_t t = tq0 + qi;
         if (t >= p.S) continue;
         const int n = st->cnt[par][qi];
@@ -831,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb_load(rb, buf, n, etid);
           RegCut c{0u, 0xFFFFFFFFu, false, n};
           if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
-          kept = rb_compact(rb, n, c, all, st->ccnt, etid, bar_id, emit);
+          kept = rb_compact(rb, n, c, all, st->scan, etid, bar_id, emit);
         } else {
           Cut cut{0u, 0xFFFFFFFFu};
           if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
@@ -861,11 +901,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bars->abort = 1;
     }
   }
-
   tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  named_bar(kExitBar, kThreads);
+  }
 }
 
 // ------------------------------------------------------------------------
@@ -876,7 +914,8 @@ static void fill_variant(ScoreVariant* v) {
   using C = Cfg<H, D, FP8>;
   v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8>);
   v->queries_per_block = C::QB;
-  v->queries_per_wg = C::NQA;
+  v->queries_per_wg = C::NQW;
+  v->groups = kEpiGroups;
   v->q_box_rows = C::BN;
   v->box_elems = C::BOX_ELEMS;
   v->smem_bytes = C::SMEM_BYTES;
