@@ -66,6 +66,9 @@ struct Plan {
   int32_t grid;
   int32_t cap;
   size_t kp_bytes;   // pooled keys (POOLED only)
+  size_t pq_bytes;   // per-query certificate terms (pruning only)
+  size_t kn_bytes;   // key norms (pruning only)
+  bool prune;
   size_t cand_bytes;
   size_t ws_bytes;
 };
@@ -74,7 +77,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
   if (!p) return INDEXER_EINVAL;
-  if (p->S < 0 || p->T < 1 || p->q_pos0 < 0 || p->K < 1 || p->flags != 0 || p->reserved != 0)
+  if (p->S < 0 || p->T < 1 || p->q_pos0 < 0 || p->K < 1 || (p->flags & ~INDEXER_FLAG_PRUNE) != 0 ||
+      p->reserved != 0)
     return INDEXER_EINVAL;
   if (p->visibility < INDEXER_VIS_TOKEN || p->visibility > INDEXER_VIS_POOLED) return INDEXER_EINVAL;
   if (p->dtype != INDEXER_BF16 && p->dtype != INDEXER_FP8_E4M3) return INDEXER_EINVAL;
@@ -111,7 +115,11 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
   pl->kp_bytes = p->visibility == INDEXER_VIS_POOLED
                      ? align256(static_cast<size_t>(pl->n_keys) * p->D * 2)
                      : 0;
-  pl->ws_bytes = kStatusBytes + pl->kp_bytes + align256(pl->cand_bytes);
+  pl->prune = (p->flags & INDEXER_FLAG_PRUNE) != 0;
+  if (pl->prune && (p->H < 2 * kPruneR || p->D % 32 != 0 || p->D > 128)) return INDEXER_EUNSUPPORTED;
+  pl->pq_bytes = pl->prune ? align256(static_cast<size_t>(p->S) * (kPruneR + 2) * sizeof(float)) : 0;
+  pl->kn_bytes = pl->prune ? align256(static_cast<size_t>(pl->n_keys) * sizeof(float)) : 0;
+  pl->ws_bytes = kStatusBytes + pl->kp_bytes + pl->pq_bytes + pl->kn_bytes + align256(pl->cand_bytes);
   return INDEXER_OK;
 }
 
@@ -194,8 +202,11 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   void* kp = ws + kStatusBytes;
-  uint2* cand = reinterpret_cast<uint2*>(ws + kStatusBytes + pl.kp_bytes);
-  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), stream) != cudaSuccess) return INDEXER_ECUDA;
+  float* pq = reinterpret_cast<float*>(ws + kStatusBytes + pl.kp_bytes);
+  float* knorm = reinterpret_cast<float*>(ws + kStatusBytes + pl.kp_bytes + pl.pq_bytes);
+  uint2* cand = reinterpret_cast<uint2*>(ws + kStatusBytes + pl.kp_bytes + pl.pq_bytes + pl.kn_bytes);
+  // status word and the three pruning counters (bytes 0, 8, 16, 24) start at zero
+  if (cudaMemsetAsync(status, 0, 32, stream) != cudaSuccess) return INDEXER_ECUDA;
   if (p->S == 0) return INDEXER_OK;
 
   const void* keys = k;
@@ -230,6 +241,13 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   sp.out_score = out_score;
   sp.cand = cand;
   sp.status = status;
+  sp.prune = pl.prune ? 1 : 0;
+  sp.pq = pq;
+  sp.knorm = knorm;
+  sp.counters = reinterpret_cast<unsigned long long*>(ws + 8);
+  if (pl.prune && launch_prune_setup(q, w, q_scale, fp8, p->S, p->H, p->D, keys, pl.n_keys, pq, knorm,
+                                     stream) != cudaSuccess)
+    return INDEXER_ECUDA;
 
   if (cudaFuncSetAttribute(pl.var.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.var.smem_bytes) !=
       cudaSuccess)
@@ -258,6 +276,17 @@ indexer_status indexer_pair_overlap(const int32_t* idx, const int32_t* len, int6
   if (!idx || !len || !out_shared) return INDEXER_EINVAL;
   if (launch_pair_overlap(idx, len, S / 2, width, out_shared, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return INDEXER_ECUDA;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_read_prune_counters(void* workspace, uint64_t* counts, void* stream) {
+  if (!workspace || !counts) return INDEXER_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned long long v[3] = {0, 0, 0};
+  if (cudaMemcpyAsync(v, static_cast<uint8_t*>(workspace) + 8, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return INDEXER_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return INDEXER_ECUDA;
+  for (int i = 0; i < 3; ++i) counts[i] = v[i];
   return INDEXER_OK;
 }
 

@@ -12,6 +12,9 @@ namespace hwr {
 constexpr uint32_t kStatusWaitTimeout = 1u;
 constexpr uint32_t kStatusOverflow = 2u;
 
+// Heads the pruning certificate keeps exactly (the first kPruneR of each query).
+constexpr int kPruneR = 16;
+
 // Arguments of the scoring + top-K kernel (one launch per indexer call).
 struct ScoreParams {
   int64_t S;          // query rows
@@ -32,6 +35,10 @@ struct ScoreParams {
   float* out_score;      // [S, width] or null
   uint2* cand;           // candidate buffers: [grid][groups][queries per group][cap]
   uint32_t* status;      // device status word
+  int32_t prune;               // 1: screen keys with the certificate before the full head sum
+  const float* pq;             // [S][kPruneR + 2]: folded weights wt[0..r), Ceff, sum |w||q|
+  const float* knorm;          // [n_keys]: |k_i| in the kernel's domain, rounded up
+  unsigned long long* counters;  // [3]: pairs screened, bounded below the threshold, skipped
 };
 
 // Per-variant launch facts, filled by the kernel's translation unit.
@@ -58,6 +65,9 @@ inline int candidate_capacity(int ksel) {
 
 cudaError_t launch_pool_keys(const void* k, int64_t n_pools, int D, const void* coef, int ratio, void* out,
                              cudaStream_t stream);
+cudaError_t launch_prune_setup(const void* q, const float* w, const float* q_scale, bool fp8, int64_t S, int H,
+                               int D, const void* keys, int64_t n_keys, float* pq, float* knorm,
+                               cudaStream_t stream);
 cudaError_t launch_pair_overlap(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
                                 int32_t* out, cudaStream_t stream);
 

@@ -1,0 +1,184 @@
+// prune.cu -- set-up of the lossless pruning stage.
+//
+// "DoSA: Dots Sparse Attention", 核心方法 / 方法步骤详情 (core method): a key
+// is skipped when a cheap upper bound U_i of its score lies below a lower
+// bound of the query's K-th score; the result must equal unpruned top-K.
+// Here the scoring kernel keeps the first kPruneR heads of every query exactly
+// and folds each other head h onto an anchor j among them, with
+// beta = [q_h.q_j]_+ / |q_j|^2 and d_h = q_h - beta q_j:
+//   w_h > 0:  w_h [q_h.k]_+ <= w_h beta [q_j.k]_+ + w_h |d_h| |k|
+//   w_h < 0:  w_h [q_h.k]_+ <= w_h beta [q_j.k]_+ + |w_h| |d_h| |k|
+// (ReLU subadditivity, positive homogeneity and Cauchy-Schwarz, the same
+// page's background section), so
+//   U_i = sum_{j < r} wt_j [a_j]_+ + Ceff |k_i|,
+//   wt_j = w_j + sum_{h -> j} w_h beta_h,  Ceff = sum_h |w_h| |d_h| + margin.
+// Everything is in the kernel's own domain: for FP8, q and k are the e4m3
+// codes the MMA multiplies, w already carries the q scale, and the key scale
+// multiplies U after the sum exactly as it multiplies the score.
+//
+// The margin covers the MMA's accumulation error and the FP32 rounding of
+// both the score and U: 2^-11 * |k| * sum_h |w_h| |q_h|.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace hwr {
+
+__device__ __forceinline__ float load_q_elem(const void* q, bool fp8, size_t i) {
+  if (fp8) {
+    __nv_fp8_e4m3 v;
+    v.__x = static_cast<const uint8_t*>(q)[i];
+    return static_cast<float>(v);
+  }
+  return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(q)[i]) << 16);
+}
+
+__device__ __forceinline__ float warp_sum_f32(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFullMask, v, o);
+  return v;
+}
+
+// Slightly enlarges a non-negative float so that it bounds the exact value the
+// FP32 computation approximated (relative 2^-18 covers a few roundings).
+__device__ __forceinline__ float round_up_pos(float x) { return x * (1.0f + 0x1p-18f) + 0x1p-100f; }
+
+// One warp per query row t: out[t] = {wt[0..r), Ceff}.  Requires D % 32 == 0
+// and D <= 128 (four values per lane), H <= 64.
+__global__ void prune_prep_kernel(const void* __restrict__ q, const float* __restrict__ w,
+                                  const float* __restrict__ q_scale, bool fp8, int64_t S, int H, int D,
+                                  float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  __shared__ float wt_s[8][kPruneR];
+  float* wt = wt_s[threadIdx.x >> 5];
+  const int per = D / 32;  // values per lane
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(warps) + (threadIdx.x >> 5); t < S;
+       t += static_cast<int64_t>(gridDim.x) * warps) {
+    const size_t qbase = static_cast<size_t>(t) * H * D;
+    // kept heads in registers: head j, dims lane + 32 m
+    float kept[kPruneR][4];
+    float nkept[kPruneR];
+    float wsum = 0.f;  // sum_h |w_h| |q_h|, rounded up
+#pragma unroll
+    for (int j = 0; j < kPruneR; ++j) {
+      float ss = 0.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        kept[j][m] = m < per ? load_q_elem(q, fp8, qbase + static_cast<size_t>(j) * D + lane + 32 * m) : 0.f;
+        ss = fmaf(kept[j][m], kept[j][m], ss);
+      }
+      nkept[j] = round_up_pos(sqrtf(warp_sum_f32(ss)));
+      float wj = w[t * H + j];
+      if (fp8) wj *= q_scale[t * H + j];
+      if (lane == 0) wt[j] = wj;
+      wsum += fabsf(wj) * nkept[j];
+    }
+    __syncwarp();
+    float C = 0.f;
+    for (int h = kPruneR; h < H; ++h) {
+      float v[4];
+      float ss = 0.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        v[m] = m < per ? load_q_elem(q, fp8, qbase + static_cast<size_t>(h) * D + lane + 32 * m) : 0.f;
+        ss = fmaf(v[m], v[m], ss);
+      }
+      const float nh = round_up_pos(sqrtf(warp_sum_f32(ss)));
+      float wh = w[t * H + h];
+      if (fp8) wh *= q_scale[t * H + h];
+      wsum += fabsf(wh) * nh;
+      // anchor: the kept head with the largest positive projection
+      int best = -1;
+      float best_proj = 0.f, best_dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < kPruneR; ++j) {
+        float dd = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) dd = fmaf(v[m], kept[j][m], dd);
+        dd = warp_sum_f32(dd);
+        const float proj = nkept[j] > 0.f ? dd / nkept[j] : 0.f;
+        if (dd > 0.f && proj > best_proj) {
+          best = j;
+          best_proj = proj;
+          best_dot = dd;
+        }
+      }
+      float beta = 0.f, nd = nh;
+      if (best >= 0) {
+        // any beta >= 0 gives a valid bound once |d| is measured for that beta
+        float nj2 = 0.f;
+#pragma unroll
+        for (int j = 0; j < kPruneR; ++j)
+          if (j == best) nj2 = nkept[j] * nkept[j];
+        beta = best_dot / nj2;
+        float ds = 0.f;
+#pragma unroll
+        for (int j = 0; j < kPruneR; ++j)
+          if (j == best) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const float d = fmaf(-beta, kept[j][m], v[m]);
+              ds = fmaf(d, d, ds);
+            }
+          }
+        nd = round_up_pos(sqrtf(warp_sum_f32(ds)));
+        // the FP32 residual d differs from q_h - beta q_j by at most one
+        // rounding per component
+        nd += 0x1p-20f * (nh + beta * sqrtf(nj2));
+        if (lane == 0) wt[best] += wh * beta;
+      }
+      C += fabsf(wh) * nd;
+      __syncwarp();
+    }
+    __syncwarp();
+    const float ceff = round_up_pos(round_up_pos(C) + 0x1p-11f * wsum);
+    float* o = out + static_cast<size_t>(t) * (kPruneR + 2);
+    if (lane < kPruneR) o[lane] = wt[lane];
+    if (lane == 0) {
+      o[kPruneR] = ceff;
+      o[kPruneR + 1] = wsum;
+    }
+    __syncwarp();
+  }
+}
+
+// norms[i] = |k_i| (kernel domain: bf16 values or e4m3 codes), rounded up.
+__global__ void key_norms_kernel(const void* __restrict__ k, bool fp8, int64_t n, int D, float* __restrict__ norms) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(warps) + (threadIdx.x >> 5); i < n;
+       i += static_cast<int64_t>(gridDim.x) * warps) {
+    float ss = 0.f;
+    for (int d = lane; d < D; d += 32) {
+      const float x = load_q_elem(k, fp8, static_cast<size_t>(i) * D + d);
+      ss = fmaf(x, x, ss);
+    }
+    ss = warp_sum_f32(ss);
+    if (lane == 0) norms[i] = round_up_pos(sqrtf(ss));
+  }
+}
+
+cudaError_t launch_prune_setup(const void* q, const float* w, const float* q_scale, bool fp8, int64_t S, int H,
+                               int D, const void* keys, int64_t n_keys, float* pq, float* knorm,
+                               cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int threads = 256;  // 8 warps
+  if (S > 0) {
+    int64_t blocks = (S + 7) / 8;
+    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+    prune_prep_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(q, w, q_scale, fp8, S, H, D, pq);
+  }
+  if (n_keys > 0) {
+    int64_t blocks = (n_keys + 7) / 8;
+    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+    key_norms_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(keys, fp8, n_keys, D, knorm);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hwr

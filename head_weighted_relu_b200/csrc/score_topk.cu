@@ -63,6 +63,7 @@ struct WgState {
   uint32_t red[16];      // reduction scratch
   int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
   int32_t scan[4];       // per-warp totals of a register-resident compaction
+  float pq[NQ][kPruneR + 4];  // pruning: folded weights of the kept heads, then Ceff
 };
 
 template <int STAGES>
@@ -141,6 +142,69 @@ __device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float
   for (int qq = 0; qq < QPC; ++qq) {
     // four independent packed partial sums (heads h mod 8 in pairs) keep the
     // FMA dependency chains short
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                     make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int h = 0; h < H; h += 4) {
+      const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
+      const float2 r01 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f),
+                                     fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f));
+      const float2 r23 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f),
+                                     fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f));
+      const int c = (h >> 2) & 1;
+      acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
+      acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
+    }
+    s[qq] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+  }
+}
+
+// Score with the pruning certificate ("DoSA: Dots Sparse Attention", 核心方法):
+// U = sum_{j<16} wt_j max(acc_j, 0) + Ceff |k| bounds the score from above;
+// when U is below the query's running threshold for all 32 keys of the warp,
+// the full head sum is skipped and the keys cannot become candidates.
+template <int H, int QPC, bool FP8, int NQ>
+__device__ __forceinline__ void score_chunk_pruned(const uint32_t (&r)[64], const float* w, float* s,
+                                                   const WgState<NQ>* st, int qi0, int32_t key, float ks, float kn,
+                                                   int lane, unsigned long long& screened,
+                                                   unsigned long long& bounded, unsigned long long& skipped) {
+#pragma unroll
+  for (int qq = 0; qq < QPC; ++qq) {
+    const int qi = qi0 + qq;
+    const float* wt = st->pq[qi];
+    float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int h = 0; h < kPruneR; h += 4) {
+      const float4 wv = *reinterpret_cast<const float4*>(wt + h);
+      const float2 r01 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f),
+                                     fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f));
+      const float2 r23 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f),
+                                     fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f));
+      u0 = __ffma2_rn(make_float2(wv.x, wv.y), r01, u0);
+      u1 = __ffma2_rn(make_float2(wv.z, wv.w), r23, u1);
+    }
+    float u = (u0.x + u0.y) + (u1.x + u1.y);
+    u = fmaf(wt[kPruneR], kn, u);
+    u += fabsf(u) * 0x1p-20f;
+    if (FP8) {
+      u *= ks;
+      u += fabsf(u) * 0x1p-20f;
+    }
+    u = __fadd_rn(u, 0.f);  // -0 -> +0, as for scores
+    const bool vis = key < st->nvis[qi];
+    const bool skip = !vis || ordered_key(u) < st->thr[qi];
+    const uint32_t vb = __ballot_sync(kFullMask, vis);
+    const uint32_t bb = __ballot_sync(kFullMask, vis && skip);
+    const bool all_skip = __all_sync(kFullMask, skip);
+    if (lane == 0) {
+      screened += static_cast<unsigned long long>(__popc(vb));
+      bounded += static_cast<unsigned long long>(__popc(bb));
+      if (all_skip) skipped += static_cast<unsigned long long>(__popc(vb));
+    }
+    if (all_skip) {
+      s[qq] = -3.0e38f;
+      continue;
+    }
     float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                      make_float2(0.f, 0.f)};
 #pragma unroll
@@ -712,6 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t af_ph = 0u;
     int par = 0;
     bool failed = false;
+    unsigned long long n_screened = 0ull, n_bounded = 0ull, n_skipped = 0ull;  // pruning counters (lane 0)
     for (int r = 0; !failed; ++r) {
       const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
       if (b < 0) break;
@@ -729,6 +794,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         wsm[i] = v;
       }
+      if (p.prune) {
+        for (int i = etid; i < NQW * (kPruneR + 2); i += kBM) {
+          const int qi = i / (kPruneR + 2), c = i % (kPruneR + 2);
+          const int64_t t = tq0 + qi;
+          st->pq[qi][c] = t < p.S ? p.pq[t * (kPruneR + 2) + c] : 0.f;
+        }
+      }
       if (etid < NQW) {
         const int64_t t = tq0 + etid;
         st->nvis[etid] = t < p.S ? n_visible(p, p.q_pos0 + t) : 0;
@@ -745,6 +817,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s[NQW];
 #pragma unroll
         for (int qi = 0; qi < NQW; ++qi) s[qi] = 0.f;
+        const int32_t key = j * kBM + etid;
+        float ks = 1.f, kn = 0.f;
+        if constexpr (FP8) ks = key < p.n_keys ? p.k_scale[key] : 0.f;
+        if (p.prune) kn = key < p.n_keys ? p.knorm[key] : 0.f;
         if (ok) {
           tc_fence_after();
           uint32_t ra[64];
@@ -759,12 +835,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               __syncwarp();
               if (lane == 0) mbar_arrive(&bars->accempty[acc]);
             }
-            score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
+            bool pruned_path = false;
+            if constexpr (H >= 2 * kPruneR) {  // the host rejects pruning for fewer heads
+              if (p.prune) {
+                score_chunk_pruned<H, C::QPC, FP8, NQW>(ra, wsm + c * 64, s + c * C::QPC, st, c * C::QPC, key,
+                                                       ks, kn, lane, n_screened, n_bounded, n_skipped);
+                pruned_path = true;
+              }
+            }
+            if (!pruned_path) score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
           }
         }
-        const int32_t key = j * kBM + etid;
         if constexpr (FP8) {
-          const float ks = key < p.n_keys ? p.k_scale[key] : 0.f;
 #pragma unroll
           for (int qi = 0; qi < NQW; ++qi) s[qi] *= ks;
         }
@@ -899,6 +981,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (failed && etid == 0) {
       atomicOr(p.status, kStatusWaitTimeout);
       bars->abort = 1;
+    }
+    if (p.prune && lane == 0) {
+      atomicAdd(&p.counters[0], n_screened);
+      atomicAdd(&p.counters[1], n_bounded);
+      atomicAdd(&p.counters[2], n_skipped);
     }
   }
   tc_fence_before();

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libhwr_indexer.so")
 
 TOKEN, COMPRESSED, POOLED = 0, 1, 2
 BF16, FP8_E4M3 = 0, 1
+FLAG_PRUNE = 1
 
 STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
                 3: "INDEXER_EUNSUPPORTED", 4: "INDEXER_ECUDA", 5: "INDEXER_EDEVICE"}
@@ -28,7 +29,8 @@ STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
 # every symbol include/hwr_indexer.h declares
 EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_topk_noalloc",
            "indexer_pool_keys",
-           "indexer_pair_overlap", "indexer_read_status", "indexer_status_string",
+           "indexer_pair_overlap", "indexer_read_status", "indexer_read_prune_counters",
+           "indexer_status_string",
            "indexer_abi_version")
 
 
@@ -62,6 +64,7 @@ def _load():
     lib.indexer_pool_keys.argtypes = [vp, i64, i32, vp, i32, vp, vp]
     lib.indexer_pair_overlap.argtypes = [vp, vp, i64, i32, vp, vp]
     lib.indexer_read_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    lib.indexer_read_prune_counters.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), vp]
     lib.indexer_status_string.argtypes = [ctypes.c_int]
     lib.indexer_status_string.restype = ctypes.c_char_p
     lib.indexer_abi_version.argtypes = []
@@ -89,11 +92,12 @@ def _check(fn, status):
         raise IndexerError(fn, status)
 
 
-def make_problem(S, T, H, D, K, visibility=TOKEN, ratio=1, dtype=BF16, q_pos0=0) -> Problem:
+def make_problem(S, T, H, D, K, visibility=TOKEN, ratio=1, dtype=BF16, q_pos0=0,
+                 prune=False) -> Problem:
     if isinstance(dtype, str):
         dtype = {"bf16": BF16, "fp8": FP8_E4M3}[dtype]
     return Problem(S=S, T=T, H=H, D=D, q_pos0=q_pos0, visibility=visibility, ratio=ratio,
-                   K=K, dtype=dtype, flags=0, reserved=0)
+                   K=K, dtype=dtype, flags=FLAG_PRUNE if prune else 0, reserved=0)
 
 
 def indexer_out_width(problem: Problem) -> int:
@@ -145,6 +149,15 @@ def indexer_read_status(workspace, stream=None) -> int:
     return f.value
 
 
+def indexer_read_prune_counters(workspace, stream=None):
+    """(pairs screened, pairs bounded below the threshold, pairs skipped) of the
+    last call that used `workspace`."""
+    c = (ctypes.c_uint64 * 3)()
+    _check("indexer_read_prune_counters", _lib.indexer_read_prune_counters(
+        _ptr(workspace), c, _stream(stream)))
+    return tuple(int(x) for x in c)
+
+
 def indexer_abi_version() -> int:
     return _lib.indexer_abi_version()
 
@@ -172,8 +185,8 @@ def allocate(problem: Problem, device, with_scores=False):
 
 
 def topk(q, k, w, K, visibility=TOKEN, ratio=1, q_pos0=0, q_scale=None, k_scale=None,
-         pool_coef=None, with_scores=False, stream=None, buffers=None):
-    """Indexer top-K of every query row.
+         pool_coef=None, with_scores=False, stream=None, buffers=None, prune=False):
+    """Indexer top-K of every query row (prune=True: the lossless pruning stage).
 
     q [S, H, D] bf16 (or e4m3 / uint8 codes with q_scale [S, H]), k [T, D] likewise
     (k_scale [T]), w [S, H] float32.  Returns (idx [S, W] int32, len [S] int32) and,
@@ -184,7 +197,7 @@ def topk(q, k, w, K, visibility=TOKEN, ratio=1, q_pos0=0, q_scale=None, k_scale=
     fp8 = q.dtype == torch.uint8
     prob = make_problem(S=S, T=k.shape[0], H=H, D=D, K=K, visibility=visibility,
                         ratio=ratio if visibility != TOKEN else 1,
-                        dtype=FP8_E4M3 if fp8 else BF16, q_pos0=q_pos0)
+                        dtype=FP8_E4M3 if fp8 else BF16, q_pos0=q_pos0, prune=prune)
     if buffers is None:
         buffers = allocate(prob, q.device, with_scores)
     out_idx, out_len, out_score, ws = buffers

@@ -45,7 +45,7 @@ class Workload:
     dtype: str = "bf16"          # storage of q and k: "bf16" or "fp8"
     q_pos0: int = 0
     seed: int = 0
-    values: str = "gauss"        # "gauss" or "int"
+    values: str = "gauss"        # "gauss", "int", or "corr" (correlated heads, w >= 0)
 
     def problem(self) -> dict:
         return dict(S=self.S, T=self.T, H=self.H, D=self.D, K=self.K,
@@ -116,6 +116,11 @@ def generate(wl: Workload, device="cpu") -> dict:
     else:
         q = _randn((wl.S, wl.H, wl.D), gen, device)
         k = _randn((wl.T, wl.D), gen, device)
+        if wl.values == "corr":
+            # structured heads: every head of a query is one shared direction
+            # plus 1% noise (what lets a score certificate prune keys)
+            z = _randn((wl.S, 1, wl.D), gen, device)
+            q.mul_(0.01).add_(z)
         if wl.dtype == "fp8":
             out["q"], out["q_scale"] = _quantise_e4m3_rows(q)
             out["k"], out["k_scale"] = _quantise_e4m3_rows(k)
@@ -123,8 +128,8 @@ def generate(wl: Workload, device="cpu") -> dict:
             out["q"] = q.to(torch.bfloat16)
             out["k"] = k.to(torch.bfloat16)
         del q, k
-        out["w"] = (_randn((wl.S, wl.H), gen, device)
-                    * (1.0 / math.sqrt(wl.H))).to(torch.float32)
+        w = _randn((wl.S, wl.H), gen, device) * (1.0 / math.sqrt(wl.H))
+        out["w"] = (w.abs() if wl.values == "corr" else w).to(torch.float32)
     if wl.visibility == POOLED:
         c = torch.rand((wl.ratio, wl.D), generator=gen, device=device,
                        dtype=torch.float32) * 0.5

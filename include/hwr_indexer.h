@@ -80,9 +80,23 @@ typedef struct {
   int32_t ratio;      /* m for COMPRESSED / POOLED (1..16); ignored for TOKEN */
   int32_t K;          /* budget in positions; POOLED selects K/ratio pools    */
   int32_t dtype;      /* indexer_dtype                                        */
-  int32_t flags;      /* must be 0                                            */
+  int32_t flags;      /* 0, or INDEXER_FLAG_PRUNE                             */
   int32_t reserved;   /* must be 0                                            */
 } indexer_problem;
+
+/* Lossless pruning ("DoSA: Dots Sparse Attention", 核心方法 / core method:
+ * skip a key whose score upper bound U_i lies below a lower bound of the
+ * K-th score, with the top-K unchanged).  The kernel keeps the first 16 heads
+ * of every query exactly and folds each other head onto one of them:
+ *   U_i = sum_{j<16} wt_j [q_j.k_i]_+ + Ceff |k_i|  >=  s_i,
+ * wt_j = w_j + sum_{h->j} w_h beta_h,  Ceff = sum_h |w_h| |q_h - beta_h q_j|
+ * plus an FP32 safety margin.  The lower bound is the running threshold of
+ * the streaming selection, which after its first cut is the K-th score of a
+ * subset of at least K visible keys (the same page's subset bound).  A key
+ * is skipped only when U_i is below that threshold, so the result is
+ * bit-identical to the run without the flag.  Needs H >= 32, D % 32 == 0,
+ * D <= 128; adds two small set-up kernels and workspace. */
+enum { INDEXER_FLAG_PRUNE = 1 };
 
 /* Row width of out_idx / out_score: K, or K + ratio - 1 for POOLED (2,051 for
  * K = 2,048 and pools of 4; KPool §2, "size index buffers to 2,051").
@@ -172,6 +186,16 @@ indexer_status indexer_pair_overlap(const int32_t* idx, const int32_t* len,
  * buffer would have overflowed (never expected; the result is not valid).
  * Also clears the word.  Host pointer `flags`. */
 indexer_status indexer_read_status(void* workspace, int32_t* flags, void* stream);
+
+/* Synchronises `stream`, then reads the pruning counters of the last
+ * indexer_topk call that used `workspace` into counts[0..2] (host array):
+ *   counts[0]  visible (query, key) pairs screened by the certificate,
+ *   counts[1]  pairs whose bound was below the query's running threshold
+ *              (the per-key pruning rate is counts[1] / counts[0]),
+ *   counts[2]  pairs whose full head sum was skipped: all 32 keys of their
+ *              warp were bounded out (the work actually saved).
+ * All zero without INDEXER_FLAG_PRUNE. */
+indexer_status indexer_read_prune_counters(void* workspace, uint64_t* counts, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* indexer_status_string(indexer_status s);
