@@ -101,10 +101,10 @@ def dist_init():
     return world, rank, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -112,6 +112,11 @@ def max_over_ranks(x: float, world: int) -> float:
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
+
+
+def rank_workload(wl, rank):
+    """Each rank's independent problem: the workload's shape, its own seed."""
+    return wl.scaled(seed=wl.seed + 1000 * rank)
 
 
 def flops_per_pair(wl):
@@ -194,7 +199,7 @@ def main():
     from head_weighted_relu_b200 import indexer as I
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl_r = wl.scaled(seed=wl.seed + 1000 * rank)
+    wl_r = rank_workload(wl, rank)
     inp = W.generate(wl_r, dev)
     prob = I.make_problem(wl.S, wl.T, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype, wl.q_pos0)
     bufs = I.allocate(prob, dev)
