@@ -35,6 +35,8 @@
 // only enter the final top-K with a score strictly above v: the threshold is
 // exact for the tie rule, and every candidate the final select sees is kept
 // or rejected exactly as a full sort of the score row would.
+#pragma once
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -236,7 +238,7 @@ struct SelResult {
 // entries with e.x == fval when `filt`.  `total` = entries passing the filter.
 // MSB-first radix select with 11-bit digits, starting below the bits that all
 // entries share.
-__device__ SelResult wg_radix_select(const uint2* buf, int n, uint32_t rank, bool idx_field, bool filt,
+__device__ inline SelResult wg_radix_select(const uint2* buf, int n, uint32_t rank, bool idx_field, bool filt,
                                      uint32_t fval, uint32_t total, uint32_t* hist, uint32_t* red,
                                      int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
@@ -326,7 +328,7 @@ struct Cut {
 };
 
 // Exact top-`ksel` of buf[0, n) under (higher ordered score, then lower index).
-__device__ Cut wg_topk_cut(const uint2* buf, int n, uint32_t ksel, uint32_t* hist, uint32_t* red, int etid,
+__device__ inline Cut wg_topk_cut(const uint2* buf, int n, uint32_t ksel, uint32_t* hist, uint32_t* red, int etid,
                            int bar_id) {
   const SelResult s1 = wg_radix_select(buf, n, ksel, false, false, 0u, static_cast<uint32_t>(n), hist, red,
                                        etid, bar_id);
@@ -409,7 +411,7 @@ __device__ __forceinline__ uint32_t rb_field(const RegBuf& b, int r, bool idx_fi
 // Largest and smallest ranked value over the valid entries (only those whose
 // ordered score equals fval when `filt`).  The next pass's barriers order the
 // reuse of `red`.
-__device__ void rb_maxmin(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t& mx,
+__device__ inline void rb_maxmin(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t& mx,
                           uint32_t& mn, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
   const int base = etid * kRegEntries;
@@ -444,7 +446,7 @@ struct Digit {
 // whose bits [lo, 32) equal prefix's.  Bin b of the histogram sits at word
 // ((b % per) << 7) + b / per, so the 128 owner threads, each summing `per`
 // consecutive bins, read distinct banks.
-__device__ Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t prefix, int lo,
+__device__ inline Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t prefix, int lo,
                          int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
   const int base = etid * kRegEntries;
@@ -512,7 +514,7 @@ struct RegCut {
 // index), starting below the bits every entry shares.  With `approx`, stops
 // after the first pass if keeping the whole digit that holds the ksel-th entry
 // keeps at most `room` entries: a safe lower bound for a running threshold.
-__device__ RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int room, uint32_t* hist,
+__device__ inline RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int room, uint32_t* hist,
                          uint32_t* red, int etid, int bar_id) {
   uint32_t mx, mn;
   rb_maxmin(b, n, false, false, 0u, mx, mn, red, etid, bar_id);
@@ -993,11 +995,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ------------------------------------------------------------------------
-// Variant table.
-// ------------------------------------------------------------------------
+
+// Launch facts of one compiled variant.
 template <int H, int D, bool FP8>
-static void fill_variant(ScoreVariant* v) {
+void fill_variant(ScoreVariant* v) {
   using C = Cfg<H, D, FP8>;
   v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8>);
   v->queries_per_block = C::QB;
@@ -1007,29 +1008,6 @@ static void fill_variant(ScoreVariant* v) {
   v->box_elems = C::BOX_ELEMS;
   v->smem_bytes = C::SMEM_BYTES;
   v->threads = kThreads;
-}
-
-bool score_variant(int H, int D, bool fp8, ScoreVariant* v) {
-#define HWR_VARIANT(h, d, f)           \
-  if (H == h && D == d && fp8 == f) { \
-    fill_variant<h, d, f>(v);          \
-    return true;                       \
-  }
-  HWR_VARIANT(4, 64, false)
-  HWR_VARIANT(4, 128, false)
-  HWR_VARIANT(8, 64, false)
-  HWR_VARIANT(8, 128, false)
-  HWR_VARIANT(16, 64, false)
-  HWR_VARIANT(16, 128, false)
-  HWR_VARIANT(32, 64, false)
-  HWR_VARIANT(32, 128, false)
-  HWR_VARIANT(64, 64, false)
-  HWR_VARIANT(64, 128, false)
-  HWR_VARIANT(16, 128, true)
-  HWR_VARIANT(32, 128, true)
-  HWR_VARIANT(64, 128, true)
-#undef HWR_VARIANT
-  return false;
 }
 
 }  // namespace hwr

@@ -1,0 +1,7 @@
+// One compiled variant of the scoring kernel (heads 16, head dim 64, BF16).
+// Variants live in separate translation units so that they compile in parallel.
+#include "score_topk.cuh"
+
+namespace hwr {
+void fill_variant_bf16_h16_d64(ScoreVariant* v) { fill_variant<16, 64, false>(v); }
+}  // namespace hwr

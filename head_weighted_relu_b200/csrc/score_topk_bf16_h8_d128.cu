@@ -1,0 +1,7 @@
+// One compiled variant of the scoring kernel (heads 8, head dim 128, BF16).
+// Variants live in separate translation units so that they compile in parallel.
+#include "score_topk.cuh"
+
+namespace hwr {
+void fill_variant_bf16_h8_d128(ScoreVariant* v) { fill_variant<8, 128, false>(v); }
+}  // namespace hwr

@@ -73,8 +73,8 @@ typedef enum {
 typedef struct {
   int64_t S;          /* query rows                                           */
   int64_t T;          /* key rows: tokens (TOKEN, POOLED) or compressed keys  */
-  int32_t H;          /* indexer heads: 4, 8, 16, 32 or 64                    */
-  int32_t D;          /* head dim: 64 or 128 (BF16), 128 (FP8)                */
+  int32_t H;          /* indexer heads (see D for the compiled pairs)         */
+  int32_t D;          /* (H, D): BF16 (4,64) (8,128) (16,64) (32,128) (64,64) (64,128); FP8 (32,128) (64,128) */
   int64_t q_pos0;     /* global position of query row 0 (g = q_pos0 + t)      */
   int32_t visibility; /* indexer_visibility                                   */
   int32_t ratio;      /* m for COMPRESSED / POOLED (1..16); ignored for TOKEN */
