@@ -6,7 +6,7 @@
 
 #include <mutex>
 
-#include "../../include/hwr_indexer.h"
+#include "hwr_indexer.h"
 #include "internal.h"
 
 namespace hwr {
@@ -92,7 +92,8 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
     if (p->K % ratio != 0) return INDEXER_EINVAL;
     if (p->dtype != INDEXER_BF16) return INDEXER_EUNSUPPORTED;
   }
-  if (!score_variant(p->H, p->D, p->dtype == INDEXER_FP8_E4M3, &pl->var)) return INDEXER_EUNSUPPORTED;
+  if (!score_variant(p->H, p->D, p->dtype == INDEXER_FP8_E4M3, (p->flags & INDEXER_FLAG_PRUNE) != 0, &pl->var))
+    return INDEXER_EUNSUPPORTED;
   pl->n_keys = p->visibility == INDEXER_VIS_POOLED ? p->T / ratio : p->T;
   pl->ksel = p->visibility == INDEXER_VIS_POOLED ? p->K / ratio : p->K;
   if (pl->ksel > (1 << 20)) return INDEXER_EUNSUPPORTED;

@@ -53,14 +53,19 @@ struct ScoreVariant {
   int threads;
 };
 
-// Returns false when (H, D, fp8) has no compiled variant.
-bool score_variant(int H, int D, bool fp8, ScoreVariant* out);
+// Returns false when (H, D, fp8, prune) has no compiled variant.
+bool score_variant(int H, int D, bool fp8, bool prune, ScoreVariant* out);
 
 // Candidate-buffer capacity per query for a selection budget of ksel keys.
 inline int candidate_capacity(int ksel) {
-  // room for the budget, plus at least as much again for new candidates
-  int c = ((2 * ksel + 127) / 128) * 128;
-  return c < ksel + 256 ? ((ksel + 256 + 127) / 128) * 128 : c;
+  // the budget plus as much again for new candidates, and up to four times the
+  // budget while that still fits the register-resident selection (4,096):
+  // fewer cuts for small budgets
+  auto r128 = [](int x) { return ((x + 127) / 128) * 128; };
+  int c = r128(2 * ksel);
+  const int wide = r128(4 * ksel);
+  if (wide <= 4096 && wide > c) c = wide;
+  return c < ksel + 256 ? r128(ksel + 256) : c;
 }
 
 cudaError_t launch_pool_keys(const void* k, int64_t n_pools, int D, const void* coef, int ratio, void* out,

@@ -13,7 +13,7 @@
 // cudaGetSymbolAddress, which is the only value ever handed to a kernel.
 #include <mutex>
 
-#include "../../include/hwr_indexer.h"
+#include "hwr_indexer.h"
 
 namespace {
 

@@ -138,6 +138,14 @@ __device__ __forceinline__ int tiles_of_block(const ScoreParams& p, int b) {
   return (n + kBM - 1) / kBM;
 }
 
+// 2 * max(x, 0) for the accumulator bits of x, computed as x + |x| on the FMA
+// pipe (exact: 2x for x >= 0, +0 otherwise).  The head weights are staged
+// halved (also exact), so w/2 * (x + |x|) rounds exactly like w * max(x, 0).
+__device__ __forceinline__ float relu2(uint32_t bits) {
+  const float x = __uint_as_float(bits);
+  return x + fabsf(x);
+}
+
 template <int H, int QPC>
 __device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float* w, float* s) {
 #pragma unroll
@@ -149,10 +157,10 @@ __device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float
 #pragma unroll
     for (int h = 0; h < H; h += 4) {
       const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
-      const float2 r01 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f),
-                                     fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f));
-      const float2 r23 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f),
-                                     fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f));
+      const float2 r01 = make_float2(relu2(r[qq * H + h + 0]),
+                                     relu2(r[qq * H + h + 1]));
+      const float2 r23 = make_float2(relu2(r[qq * H + h + 2]),
+                                     relu2(r[qq * H + h + 3]));
       const int c = (h >> 2) & 1;
       acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
       acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
@@ -178,10 +186,10 @@ __device__ __forceinline__ void score_chunk_pruned(const uint32_t (&r)[64], cons
 #pragma unroll
     for (int h = 0; h < kPruneR; h += 4) {
       const float4 wv = *reinterpret_cast<const float4*>(wt + h);
-      const float2 r01 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f),
-                                     fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f));
-      const float2 r23 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f),
-                                     fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f));
+      const float2 r01 = make_float2(relu2(r[qq * H + h + 0]),
+                                     relu2(r[qq * H + h + 1]));
+      const float2 r23 = make_float2(relu2(r[qq * H + h + 2]),
+                                     relu2(r[qq * H + h + 3]));
       u0 = __ffma2_rn(make_float2(wv.x, wv.y), r01, u0);
       u1 = __ffma2_rn(make_float2(wv.z, wv.w), r23, u1);
     }
@@ -212,10 +220,10 @@ __device__ __forceinline__ void score_chunk_pruned(const uint32_t (&r)[64], cons
 #pragma unroll
     for (int h = 0; h < H; h += 4) {
       const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
-      const float2 r01 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 0]), 0.f),
-                                     fmaxf(__uint_as_float(r[qq * H + h + 1]), 0.f));
-      const float2 r23 = make_float2(fmaxf(__uint_as_float(r[qq * H + h + 2]), 0.f),
-                                     fmaxf(__uint_as_float(r[qq * H + h + 3]), 0.f));
+      const float2 r01 = make_float2(relu2(r[qq * H + h + 0]),
+                                     relu2(r[qq * H + h + 1]));
+      const float2 r23 = make_float2(relu2(r[qq * H + h + 2]),
+                                     relu2(r[qq * H + h + 3]));
       const int c = (h >> 2) & 1;
       acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
       acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
@@ -600,7 +608,7 @@ __device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
-template <int H, int D, bool FP8>
+template <int H, int D, bool FP8, bool PRUNE>
 __global__ void __launch_bounds__(kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const ScoreParams p) {
@@ -794,13 +802,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           v = p.w[t * H + (i % H)];
           if constexpr (FP8) v *= p.q_scale[t * H + (i % H)];
         }
-        wsm[i] = v;
+        wsm[i] = 0.5f * v;  // halved: the ReLU is computed doubled (relu2)
       }
-      if (p.prune) {
+      if constexpr (PRUNE) {
         for (int i = etid; i < NQW * (kPruneR + 2); i += kBM) {
           const int qi = i / (kPruneR + 2), c = i % (kPruneR + 2);
           const int64_t t = tq0 + qi;
-          st->pq[qi][c] = t < p.S ? p.pq[t * (kPruneR + 2) + c] : 0.f;
+          const float v = t < p.S ? p.pq[t * (kPruneR + 2) + c] : 0.f;
+          st->pq[qi][c] = c < kPruneR ? 0.5f * v : v;  // kept-head weights halved, as for relu2
         }
       }
       if (etid < NQW) {
@@ -822,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t key = j * kBM + etid;
         float ks = 1.f, kn = 0.f;
         if constexpr (FP8) ks = key < p.n_keys ? p.k_scale[key] : 0.f;
-        if (p.prune) kn = key < p.n_keys ? p.knorm[key] : 0.f;
+        if constexpr (PRUNE) kn = key < p.n_keys ? p.knorm[key] : 0.f;
         if (ok) {
           tc_fence_after();
           uint32_t ra[64];
@@ -838,8 +847,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (lane == 0) mbar_arrive(&bars->accempty[acc]);
             }
             bool pruned_path = false;
-            if constexpr (H >= 2 * kPruneR) {  // the host rejects pruning for fewer heads
-              if (p.prune) {
+            if constexpr (PRUNE && H >= 2 * kPruneR) {  // the host rejects pruning for fewer heads
+              {
                 score_chunk_pruned<H, C::QPC, FP8, NQW>(ra, wsm + c * 64, s + c * C::QPC, st, c * C::QPC, key,
                                                        ks, kn, lane, n_screened, n_bounded, n_skipped);
                 pruned_path = true;
@@ -984,7 +993,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicOr(p.status, kStatusWaitTimeout);
       bars->abort = 1;
     }
-    if (p.prune && lane == 0) {
+    if (PRUNE && lane == 0) {
       atomicAdd(&p.counters[0], n_screened);
       atomicAdd(&p.counters[1], n_bounded);
       atomicAdd(&p.counters[2], n_skipped);
@@ -997,10 +1006,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
 // Launch facts of one compiled variant.
-template <int H, int D, bool FP8>
+template <int H, int D, bool FP8, bool PRUNE>
 void fill_variant(ScoreVariant* v) {
   using C = Cfg<H, D, FP8>;
-  v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8>);
+  v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8, PRUNE>);
   v->queries_per_block = C::QB;
   v->queries_per_wg = C::NQW;
   v->groups = kEpiGroups;

@@ -3,5 +3,5 @@
 #include "score_topk.cuh"
 
 namespace hwr {
-void fill_variant_bf16_h32_d128(ScoreVariant* v) { fill_variant<32, 128, false>(v); }
+void fill_variant_bf16_h32_d128(ScoreVariant* v) { fill_variant<32, 128, false, false>(v); }
 }  // namespace hwr

@@ -3,5 +3,5 @@
 #include "score_topk.cuh"
 
 namespace hwr {
-void fill_variant_bf16_h4_d64(ScoreVariant* v) { fill_variant<4, 64, false>(v); }
+void fill_variant_bf16_h4_d64(ScoreVariant* v) { fill_variant<4, 64, false, false>(v); }
 }  // namespace hwr

@@ -3,5 +3,5 @@
 #include "score_topk.cuh"
 
 namespace hwr {
-void fill_variant_fp8_h32_d128(ScoreVariant* v) { fill_variant<32, 128, true>(v); }
+void fill_variant_fp8_h32_d128(ScoreVariant* v) { fill_variant<32, 128, true, false>(v); }
 }  // namespace hwr

@@ -17,7 +17,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libhwr_indexer.so")
+# HWR_INDEXER_LIB may point at another build of the same library (same ABI)
+LIB_PATH = os.environ.get("HWR_INDEXER_LIB") or os.path.join(_HERE, "libhwr_indexer.so")
 
 TOKEN, COMPRESSED, POOLED = 0, 1, 2
 BF16, FP8_E4M3 = 0, 1
