@@ -61,7 +61,7 @@ struct WgState {
   uint32_t thr[NQ];      // a candidate is appended iff its ordered score >= thr
   int32_t cnt[2][NQ];    // candidates held, double-buffered by tile parity
   int32_t nvis[NQ];      // keys visible to each query of the group
-  int32_t wc[2][NQ][4];  // per-warp pass counts, double-buffered by tile parity
+  int4 wc[2][NQ];        // per-warp pass counts (x..w = warps 0..3), double-buffered by tile parity
   uint32_t red[16];      // reduction scratch
   int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
   int32_t scan[4];       // per-warp totals of a register-resident compaction
@@ -862,12 +862,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int qi = 0; qi < NQW; ++qi) s[qi] *= ks;
         }
         // pass flags and per-warp counts
+        uint32_t okeys[NQW], bals[NQW];
 #pragma unroll
         for (int qi = 0; qi < NQW; ++qi) {
-          const uint32_t okey = ordered_key(__fadd_rn(s[qi], 0.f));
-          const bool pass = ok && key < st->nvis[qi] && okey >= st->thr[qi];
-          const uint32_t bal = __ballot_sync(kFullMask, pass);
-          if (lane == 0) st->wc[par][qi][wq] = __popc(bal);
+          okeys[qi] = ordered_key(__fadd_rn(s[qi], 0.f));
+          const bool pass = ok && key < st->nvis[qi] && okeys[qi] >= st->thr[qi];
+          bals[qi] = __ballot_sync(kFullMask, pass);
+          if (lane == 0) reinterpret_cast<int32_t*>(&st->wc[par][qi])[wq] = __popc(bals[qi]);
         }
         if (named_bar_or(bar_id, kBM, !ok)) {
           failed = true;
@@ -878,22 +879,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // here is double-buffered by tile parity.
         const int np = par ^ 1;
         int newcnt[NQW];
+        const uint32_t lt_mask = (1u << lane) - 1u;
 #pragma unroll
         for (int qi = 0; qi < NQW; ++qi) {
-          const uint32_t okey = ordered_key(__fadd_rn(s[qi], 0.f));
-          const bool pass = key < st->nvis[qi] && okey >= st->thr[qi];
-          const uint32_t bal = __ballot_sync(kFullMask, pass);
+          const uint32_t bal = bals[qi];
           const int held = st->cnt[par][qi];
-          int prior = 0, tot = 0;
-#pragma unroll
-          for (int w2 = 0; w2 < 4; ++w2) {
-            const int cc = st->wc[par][qi][w2];
-            tot += cc;
-            prior += (w2 < wq) ? cc : 0;
-          }
-          if (pass) {
-            const int pos = held + prior + __popc(bal & ((1u << lane) - 1u));
-            cand[qi * static_cast<size_t>(p.cap) + pos] = make_uint2(okey, static_cast<uint32_t>(key));
+          const int4 wc = st->wc[par][qi];
+          const int tot = wc.x + wc.y + wc.z + wc.w;
+          const int prior = (wq > 0 ? wc.x : 0) + (wq > 1 ? wc.y : 0) + (wq > 2 ? wc.z : 0);
+          if ((bal >> lane) & 1u) {
+            const int pos = held + prior + __popc(bal & lt_mask);
+            cand[qi * static_cast<size_t>(p.cap) + pos] = make_uint2(okeys[qi], static_cast<uint32_t>(key));
           }
           newcnt[qi] = held + tot;
           if (etid == qi) st->cnt[np][qi] = held + tot;
