@@ -900,9 +900,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int qi = 0; qi < NQW; ++qi) any_full |= newcnt[qi] > p.cap - kBM;
         if (any_full) named_bar(bar_id, kBM);  // every append of this tile is visible
-#pragma unroll
+#pragma unroll 1
         for (int qi = 0; qi < NQW; ++qi) {
-          const int n = newcnt[qi];
+          int n = 0;  // newcnt[qi], read without a dynamic register index
+#pragma unroll
+          for (int k = 0; k < NQW; ++k) n = (k == qi) ? newcnt[k] : n;
           if (n > p.cap - kBM) {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
             int kept;
