@@ -820,92 +820,107 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_bar(bar_id, kBM);
 
-      for (int j = 0; j < nt; ++j) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(&bars->accfull[acc], af_ph, abort_flag, kWaitLimitNs);
-        ok = __shfl_sync(kFullMask, ok ? 1 : 0, 0) != 0;
-        af_ph ^= 1u;
-        float s[NQW];
-#pragma unroll
-        for (int qi = 0; qi < NQW; ++qi) s[qi] = 0.f;
-        const int32_t key = j * kBM + etid;
-        float ks = 1.f, kn = 0.f;
-        if constexpr (FP8) ks = key < p.n_keys ? p.k_scale[key] : 0.f;
-        if constexpr (PRUNE) kn = key < p.n_keys ? p.knorm[key] : 0.f;
-        if (ok) {
-          tc_fence_after();
-          uint32_t ra[64];
-#pragma unroll
-          for (int c = 0; c < C::CHUNKS_W; ++c) {
-            tmem_ld_x64(tbase + c * 64, ra);
-            tmem_wait_ld(ra);
-            if (c + 1 == C::CHUNKS_W) {
-              // everything this warp needs from TMEM is in registers: hand the
-              // accumulator back before the last chunk's arithmetic
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&bars->accempty[acc]);
-            }
-            bool pruned_path = false;
-            if constexpr (PRUNE && H >= 2 * kPruneR) {  // the host rejects pruning for fewer heads
-              {
-                score_chunk_pruned<H, C::QPC, FP8, NQW>(ra, wsm + c * 64, s + c * C::QPC, st, c * C::QPC, key,
-                                                       ks, kn, lane, n_screened, n_bounded, n_skipped);
-                pruned_path = true;
-              }
-            }
-            if (!pruned_path) score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
-          }
-        }
-        if constexpr (FP8) {
-#pragma unroll
-          for (int qi = 0; qi < NQW; ++qi) s[qi] *= ks;
-        }
-        // pass flags and per-warp counts
-        uint32_t okeys[NQW], bals[NQW];
-#pragma unroll
-        for (int qi = 0; qi < NQW; ++qi) {
-          okeys[qi] = ordered_key(__fadd_rn(s[qi], 0.f));
-          const bool pass = ok && key < st->nvis[qi] && okeys[qi] >= st->thr[qi];
-          bals[qi] = __ballot_sync(kFullMask, pass);
-          if (lane == 0) reinterpret_cast<int32_t*>(&st->wc[par][qi])[wq] = __popc(bals[qi]);
-        }
-        if (named_bar_or(bar_id, kBM, !ok)) {
-          failed = true;
-          break;
-        }
-        // ordered append: position = held + earlier warps + earlier lanes.  No
-        // barrier follows: every thread knows the new counts, and the state read
-        // here is double-buffered by tile parity.
-        const int np = par ^ 1;
-        int newcnt[NQW];
-        const uint32_t lt_mask = (1u << lane) - 1u;
-#pragma unroll
-        for (int qi = 0; qi < NQW; ++qi) {
-          const uint32_t bal = bals[qi];
-          const int held = st->cnt[par][qi];
-          const int4 wc = st->wc[par][qi];
-          const int tot = wc.x + wc.y + wc.z + wc.w;
-          const int prior = (wq > 0 ? wc.x : 0) + (wq > 1 ? wc.y : 0) + (wq > 2 ? wc.z : 0);
-          if ((bal >> lane) & 1u) {
-            const int pos = held + prior + __popc(bal & lt_mask);
-            cand[qi * static_cast<size_t>(p.cap) + pos] = make_uint2(okeys[qi], static_cast<uint32_t>(key));
-          }
-          newcnt[qi] = held + tot;
-          if (etid == qi) st->cnt[np][qi] = held + tot;
-        }
-        par = np;
-        // cut buffers that could not take another full tile back toward their top-K
+      // Tiles run in a tight loop that leaves when a candidate buffer is about
+      // to overflow or the block's tiles are done; the selection steps (cut of
+      // the full buffers, or the final top-K of every query) follow it, so the
+      // per-tile path carries none of their code.
+      int j = 0;
+      while (true) {
         bool any_full = false;
+        for (; j < nt; ++j) {
+          // every lane polls (no divergent branch around the wait); the phase
+          // is complete for all once any lane has seen it complete
+          bool ok = mbar_wait(&bars->accfull[acc], af_ph, abort_flag, kWaitLimitNs);
+          ok = __any_sync(kFullMask, ok);
+          af_ph ^= 1u;
+          float s[NQW];
 #pragma unroll
-        for (int qi = 0; qi < NQW; ++qi) any_full |= newcnt[qi] > p.cap - kBM;
-        if (any_full) named_bar(bar_id, kBM);  // every append of this tile is visible
+          for (int qi = 0; qi < NQW; ++qi) s[qi] = 0.f;
+          const int32_t key = j * kBM + etid;
+          float ks = 1.f, kn = 0.f;
+          if constexpr (FP8) ks = key < p.n_keys ? p.k_scale[key] : 0.f;
+          if constexpr (PRUNE) kn = key < p.n_keys ? p.knorm[key] : 0.f;
+          if (ok) {
+            tc_fence_after();
+            uint32_t ra[64];
+#pragma unroll
+            for (int c = 0; c < C::CHUNKS_W; ++c) {
+              tmem_ld_x64(tbase + c * 64, ra);
+              tmem_wait_ld(ra);
+              if (c + 1 == C::CHUNKS_W) {
+                // everything this warp needs from TMEM is in registers: hand the
+                // accumulator back before the last chunk's arithmetic
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->accempty[acc]);
+              }
+              bool pruned_path = false;
+              if constexpr (PRUNE && H >= 2 * kPruneR) {  // the host rejects pruning for fewer heads
+                {
+                  score_chunk_pruned<H, C::QPC, FP8, NQW>(ra, wsm + c * 64, s + c * C::QPC, st, c * C::QPC, key,
+                                                         ks, kn, lane, n_screened, n_bounded, n_skipped);
+                  pruned_path = true;
+                }
+              }
+              if (!pruned_path) score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
+            }
+          }
+          if constexpr (FP8) {
+#pragma unroll
+            for (int qi = 0; qi < NQW; ++qi) s[qi] *= ks;
+          }
+          // pass flags and per-warp counts
+          uint32_t okeys[NQW], bals[NQW];
+#pragma unroll
+          for (int qi = 0; qi < NQW; ++qi) {
+            okeys[qi] = ordered_key(__fadd_rn(s[qi], 0.f));
+            const bool pass = ok && key < st->nvis[qi] && okeys[qi] >= st->thr[qi];
+            bals[qi] = __ballot_sync(kFullMask, pass);
+            if (lane == 0) reinterpret_cast<int32_t*>(&st->wc[par][qi])[wq] = __popc(bals[qi]);
+          }
+          if (named_bar_or(bar_id, kBM, !ok)) {
+            failed = true;
+            break;
+          }
+          // ordered append: position = held + earlier warps + earlier lanes.  No
+          // barrier follows: every thread knows the new counts, and the state read
+          // here is double-buffered by tile parity.
+          const int np = par ^ 1;
+          int newcnt[NQW];
+          const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+          for (int qi = 0; qi < NQW; ++qi) {
+            const uint32_t bal = bals[qi];
+            const int held = st->cnt[par][qi];
+            const int4 wc = st->wc[par][qi];
+            const int tot = wc.x + wc.y + wc.z + wc.w;
+            const int prior = (wq > 0 ? wc.x : 0) + (wq > 1 ? wc.y : 0) + (wq > 2 ? wc.z : 0);
+            if ((bal >> lane) & 1u) {
+              const int pos = held + prior + __popc(bal & lt_mask);
+              cand[qi * static_cast<size_t>(p.cap) + pos] = make_uint2(okeys[qi], static_cast<uint32_t>(key));
+            }
+            newcnt[qi] = held + tot;
+            if (etid == qi) st->cnt[np][qi] = held + tot;
+          }
+          par = np;
+#pragma unroll
+          for (int qi = 0; qi < NQW; ++qi) any_full |= newcnt[qi] > p.cap - kBM;
+          if (any_full) {
+            ++j;
+            break;
+          }
+        }
+        if (failed) break;
+        // no buffer is full: the block's tiles are done and the final top-K of
+        // each query is written; otherwise the full buffers are cut back
+        const bool fin = !any_full;
+        named_bar(bar_id, kBM);  // every append and count of the last tile is visible to the group
 #pragma unroll 1
         for (int qi = 0; qi < NQW; ++qi) {
-          int n = 0;  // newcnt[qi], read without a dynamic register index
-#pragma unroll
-          for (int k = 0; k < NQW; ++k) n = (k == qi) ? newcnt[k] : n;
-          if (n > p.cap - kBM) {
+          const int n = st->cnt[par][qi];
+          const int64_t t = tq0 + qi;
+          if (fin ? t >= p.S : n <= p.cap - kBM) continue;
+          if (!fin) {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
             int kept;
             uint32_t thr;
@@ -927,64 +942,57 @@ __global__ void __launch_bounds__(kThreads, 1)
               st->cnt[par][qi] = kept;
               st->thr[qi] = thr;
             }
-            named_bar(bar_id, kBM);
-          }
-        }
-      }
-      if (failed) break;
-
-      // final selection of each query of the group, written in key order
-#pragma unroll 1
-      for (int qi = 0; qi < NQW; ++qi) {
-        const int64_t t = tq0 + qi;
-        if (t >= p.S) continue;
-        const int n = st->cnt[par][qi];
-        uint2* buf = cand + qi * static_cast<size_t>(p.cap);
-        const bool all = n <= p.ksel;
-        int32_t* orow = p.out_idx + t * p.width;
-        float* srow = p.out_score ? p.out_score + t * p.width : nullptr;
-        const int m = p.out_ratio;
-        auto emit = [&](int pos, uint32_t k, uint32_t ix) {
-          const float sc = key_to_float(k);
-          if (m == 1) {
-            orow[pos] = static_cast<int32_t>(ix);
-            if (srow) srow[pos] = sc;
           } else {
-            for (int rr = 0; rr < m; ++rr) {
-              orow[pos * m + rr] = static_cast<int32_t>(ix) * m + rr;
-              if (srow) srow[pos * m + rr] = sc;
+            uint2* buf = cand + qi * static_cast<size_t>(p.cap);
+            const bool all = n <= p.ksel;
+            int32_t* orow = p.out_idx + t * p.width;
+            float* srow = p.out_score ? p.out_score + t * p.width : nullptr;
+            const int m = p.out_ratio;
+            auto emit = [&](int pos, uint32_t k, uint32_t ix) {
+              const float sc = key_to_float(k);
+              if (m == 1) {
+                orow[pos] = static_cast<int32_t>(ix);
+                if (srow) srow[pos] = sc;
+              } else {
+                for (int rr = 0; rr < m; ++rr) {
+                  orow[pos * m + rr] = static_cast<int32_t>(ix) * m + rr;
+                  if (srow) srow[pos * m + rr] = sc;
+                }
+              }
+            };
+            int kept;
+            if (n <= kRegCap) {
+              RegBuf rb;
+              rb_load(rb, buf, n, etid);
+              RegCut c{0u, 0xFFFFFFFFu, false, n};
+              if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
+              kept = rb_compact(rb, n, c, all, st->scan, etid, bar_id, emit);
+            } else {
+              Cut cut{0u, 0xFFFFFFFFu};
+              if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
+              kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id,
+                                [&](int pos, uint2 e) { emit(pos, e.x, e.y); });
             }
+            int len = kept * m;
+            if (m > 1) {
+              const int64_t g = p.q_pos0 + t;
+              const int tail = static_cast<int>((g + 1) % m);
+              const int64_t first = g + 1 - tail;
+              for (int i = etid; i < tail; i += kBM) {
+                orow[len + i] = static_cast<int32_t>(first + i);
+                if (srow) srow[len + i] = __uint_as_float(0x7FC00000u);
+              }
+              len += tail;
+            }
+            for (int i = len + etid; i < p.width; i += kBM) {
+              orow[i] = -1;
+              if (srow) srow[i] = __uint_as_float(0x7FC00000u);
+            }
+            if (etid == 0) p.out_len[t] = len;
           }
-        };
-        int kept;
-        if (n <= kRegCap) {
-          RegBuf rb;
-          rb_load(rb, buf, n, etid);
-          RegCut c{0u, 0xFFFFFFFFu, false, n};
-          if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
-          kept = rb_compact(rb, n, c, all, st->scan, etid, bar_id, emit);
-        } else {
-          Cut cut{0u, 0xFFFFFFFFu};
-          if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
-          kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id,
-                            [&](int pos, uint2 e) { emit(pos, e.x, e.y); });
+          named_bar(bar_id, kBM);
         }
-        int len = kept * m;
-        if (m > 1) {
-          const int64_t g = p.q_pos0 + t;
-          const int tail = static_cast<int>((g + 1) % m);
-          const int64_t first = g + 1 - tail;
-          for (int i = etid; i < tail; i += kBM) {
-            orow[len + i] = static_cast<int32_t>(first + i);
-            if (srow) srow[len + i] = __uint_as_float(0x7FC00000u);
-          }
-          len += tail;
-        }
-        for (int i = len + etid; i < p.width; i += kBM) {
-          orow[i] = -1;
-          if (srow) srow[i] = __uint_as_float(0x7FC00000u);
-        }
-        if (etid == 0) p.out_len[t] = len;
+        if (fin) break;
       }
     }
     if (failed && etid == 0) {
