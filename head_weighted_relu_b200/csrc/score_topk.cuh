@@ -11,24 +11,29 @@
 // partition-merge top-K instead of materialising scores; this kernel streams
 // keys in ascending order and merges into a running selection.
 //
-// One persistent CTA per SM, 20 warps:
-//   warp 0      TMA producer: the query block's q rows once, then key tiles of
-//               128 rows through a ring of shared-memory stages;
-//   warp 1      MMA issuer: for each key tile, two accumulators
-//               acc[a][key, (query, head)] = k_tile . q_block[a]^T
+// One persistent CTA per SM, 20 warps, one query block (the queries of one
+// accumulator: 4 for 64 heads, 8 for 32, ...) at a time:
+//   warp 0      TMA producer: the block's q rows once, then key tiles of 128
+//               rows through a ring of shared-memory stages;
+//   warp 1      MMA issuer: key tile n goes to accumulator n & 1,
+//               acc[key, (query, head)] = k_tile . q_block^T
 //               (M = 128 keys = TMEM lanes, N = queries x heads <= 256 columns,
-//               K = D), tcgen05.mma with FP32 accumulation in TMEM;
-//   warps 4..19 four epilogue warpgroups, two per accumulator, each taking
-//               half of its queries.  Each thread owns one key (one TMEM
-//               lane) and, for every query of its group,
-//               reduces sum_h w[t,h] * max(acc, 0) in registers, applies the
-//               visibility mask, and appends (ordered score, key) pairs that
-//               beat the query's running threshold to a per-query candidate
-//               buffer in global memory -- in key order, so the buffer is
-//               always sorted by key index.  A buffer about to overflow is cut
-//               back to its exact top-K by a warpgroup radix select, which
-//               raises the threshold.  After the query block's last tile the
-//               same select gives the final top-K, written in key order.
+//               K = D), tcgen05.mma with FP32 accumulation in TMEM, so the
+//               next tile's product overlaps the epilogue of this one;
+//   warps 4..19 four epilogue warpgroups, each owning a quarter of the
+//               columns (whole queries).  A warpgroup keeps its queries' head
+//               weights in registers for the whole block, so the head sum
+//               reads nothing but TMEM: 16-column loads, double-buffered, and
+//               one packed FMA per pair of heads.  Each thread owns one key
+//               (one TMEM lane) and, for every query of its group, reduces
+//               sum_h w[t,h] * max(acc, 0), applies the visibility mask, and
+//               appends (ordered score, key) pairs that beat the query's
+//               running threshold to a per-query candidate buffer in global
+//               memory -- in key order, so the buffer is always sorted by key
+//               index.  A buffer about to overflow is cut back toward its
+//               top-K by a warpgroup radix select, which raises the threshold.
+//               After the block's last tile the same select gives the final
+//               top-K, written in key order.
 //
 // Keys arrive in ascending index order, so once a buffer holds the top-K of
 // the keys seen so far with K-th entry (v, i), a later key (index > i) can
@@ -86,18 +91,21 @@ struct Cfg {
   static constexpr int NBOX = ROW_BYTES / 128;          // 128-byte swizzle boxes per row
   static constexpr int BOX_ELEMS = 128 / ELEM;
   static constexpr int KSTEPS = ROW_BYTES / 32;          // MMA K steps of 32 bytes
-  static constexpr int NQA = (256 / H) < 32 ? (256 / H) : 32;  // queries per accumulator
-  static constexpr int NQW = NQA / 2;                    // queries per epilogue warpgroup
+  static constexpr int NQA = (256 / H) < 32 ? (256 / H) : 32;  // queries per accumulator = per block
+  static constexpr int QB = NQA;                         // queries per block
   static constexpr int BN = NQA * H;                     // accumulator columns = MMA N
-  static constexpr int QB = 2 * NQA;                     // queries per block
-  static constexpr int CHUNKS_W = (BN / 2) / 64;         // 64-column TMEM loads per warpgroup
-  static constexpr int QPC = 64 / H;                     // queries per 64-column load
+  static constexpr int CW = BN / 4;                      // columns (query, head) per epilogue warpgroup
+  static constexpr int NQW = CW / H;                     // queries per epilogue warpgroup
+  static constexpr int NCH = CW / 16;                    // 16-column TMEM loads per warpgroup and tile
+  static constexpr bool WREG = NQW <= 2;                 // head weights held in registers
+  static constexpr int WSM_COLS = WREG ? 16 : CW;         // columns whose weights stay in shared memory
+  static constexpr int CHAINS = NQW == 1 ? 4 : 2;        // packed partial sums per query
   static constexpr int Q_ACC_BYTES = BN * ROW_BYTES;
-  static constexpr int Q_BYTES = 2 * Q_ACC_BYTES;
+  static constexpr int Q_BYTES = Q_ACC_BYTES;
   static constexpr int K_STAGE_BYTES = kBM * ROW_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMALL_BYTES =
-      kHistBins * 4 * kEpiGroups + 2 * BN * 4 + kEpiGroups * (int)sizeof(WgState<NQW>);
+      kHistBins * 4 * kEpiGroups + BN * 4 + kEpiGroups * (int)sizeof(WgState<NQW>);
   static constexpr int AVAIL = kSmemLimit - 1024 - Q_BYTES - SMALL_BYTES - (int)sizeof(Barriers<8>);
   static constexpr int STAGES_RAW = AVAIL / K_STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
@@ -105,13 +113,14 @@ struct Cfg {
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_HIST = OFF_K + STAGES * K_STAGE_BYTES;
   static constexpr int OFF_W = OFF_HIST + kHistBins * 4 * kEpiGroups;
-  static constexpr int OFF_ST = OFF_W + 2 * BN * 4;
+  static constexpr int OFF_ST = OFF_W + BN * 4;
   static constexpr int OFF_BAR = OFF_ST + kEpiGroups * (int)sizeof(WgState<NQW>);
   static constexpr int SMEM_BYTES = 1024 + OFF_BAR + (int)sizeof(Barriers<STAGES>);
   static constexpr uint32_t IDESC = FP8 ? idesc_e4m3<kBM, BN>() : idesc_bf16<kBM, BN>();
   static_assert(H % 4 == 0 && H <= 64, "heads");
   static_assert(ROW_BYTES % 128 == 0, "row must be whole 128-byte swizzle rows");
   static_assert(BN % 128 == 0 && BN >= 128 && BN <= 256, "accumulator width");
+  static_assert(CW % 16 == 0 && CW % H == 0 && H % 2 == 0, "whole queries per group, 16-column loads");
   static_assert(STAGES >= 2, "shared memory too small for a 2-stage key ring");
   static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
   static_assert(OFF_K % 1024 == 0 && K_STAGE_BYTES % 1024 == 0 && Q_ACC_BYTES % 1024 == 0, "swizzle alignment");
@@ -146,90 +155,53 @@ __device__ __forceinline__ float relu2(uint32_t bits) {
   return x + fabsf(x);
 }
 
-template <int H, int QPC>
-__device__ __forceinline__ void score_chunk(const uint32_t (&r)[64], const float* w, float* s) {
+// Adds one 16-column TMEM chunk of the group's columns into the packed partial
+// sums: column col0 + k holds query (col0 + k) / H, head (col0 + k) % H.  Each
+// pair of heads goes through one packed FMA with the pair's halved weights
+// (wget(col) returns them as a float2); pair p of a query feeds chain
+// p % CHAINS.  Every index is a compile-time constant once the callers'
+// loops are unrolled, so the sums and register-held weights stay in registers.
+template <int H, int NQW, int CHAINS, class WGet>
+__device__ __forceinline__ void chunk_fma(const uint32_t (&r)[16], int col0, WGet wget,
+                                          float2 (&acc)[NQW][CHAINS]) {
 #pragma unroll
-  for (int qq = 0; qq < QPC; ++qq) {
-    // four independent packed partial sums (heads h mod 8 in pairs) keep the
-    // FMA dependency chains short
-    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                     make_float2(0.f, 0.f)};
-#pragma unroll
-    for (int h = 0; h < H; h += 4) {
-      const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
-      const float2 r01 = make_float2(relu2(r[qq * H + h + 0]),
-                                     relu2(r[qq * H + h + 1]));
-      const float2 r23 = make_float2(relu2(r[qq * H + h + 2]),
-                                     relu2(r[qq * H + h + 3]));
-      const int c = (h >> 2) & 1;
-      acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
-      acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
-    }
-    s[qq] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+  for (int k = 0; k < 16; k += 2) {
+    const int col = col0 + k;
+    const int qi = col / H;
+    const int ch = ((col % H) >> 1) % CHAINS;
+    acc[qi][ch] = __ffma2_rn(wget(col), make_float2(relu2(r[k]), relu2(r[k + 1])), acc[qi][ch]);
   }
 }
 
-// Score with the pruning certificate ("DoSA: Dots Sparse Attention", 核心方法):
-// U = sum_{j<16} wt_j max(acc_j, 0) + Ceff |k| bounds the score from above;
-// when U is below the query's running threshold for all 32 keys of the warp,
-// the full head sum is skipped and the keys cannot become candidates.
-template <int H, int QPC, bool FP8, int NQ>
-__device__ __forceinline__ void score_chunk_pruned(const uint32_t (&r)[64], const float* w, float* s,
-                                                   const WgState<NQ>* st, int qi0, int32_t key, float ks, float kn,
-                                                   int lane, unsigned long long& screened,
-                                                   unsigned long long& bounded, unsigned long long& skipped) {
+// The score from a query's partial sums, added in a fixed tree.
+template <int CHAINS>
+__device__ __forceinline__ float chain_total(const float2 (&a)[CHAINS]) {
+  if constexpr (CHAINS == 4)
+    return ((a[0].x + a[0].y) + (a[1].x + a[1].y)) + ((a[2].x + a[2].y) + (a[3].x + a[3].y));
+  else
+    return (a[0].x + a[0].y) + (a[1].x + a[1].y);
+}
+
+// Upper bound of a key's score from the first kPruneR heads of a query
+// ("DoSA: Dots Sparse Attention", 核心方法): U = sum_{j<16} wt_j max(acc_j, 0) +
+// Ceff |k|, widened by a few roundings; r holds the query's first 16 columns.
+template <bool FP8>
+__device__ __forceinline__ float prune_bound(const uint32_t (&r)[16], const float* wt, float ks, float kn) {
+  float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int qq = 0; qq < QPC; ++qq) {
-    const int qi = qi0 + qq;
-    const float* wt = st->pq[qi];
-    float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int h = 0; h < kPruneR; h += 4) {
-      const float4 wv = *reinterpret_cast<const float4*>(wt + h);
-      const float2 r01 = make_float2(relu2(r[qq * H + h + 0]),
-                                     relu2(r[qq * H + h + 1]));
-      const float2 r23 = make_float2(relu2(r[qq * H + h + 2]),
-                                     relu2(r[qq * H + h + 3]));
-      u0 = __ffma2_rn(make_float2(wv.x, wv.y), r01, u0);
-      u1 = __ffma2_rn(make_float2(wv.z, wv.w), r23, u1);
-    }
-    float u = (u0.x + u0.y) + (u1.x + u1.y);
-    u = fmaf(wt[kPruneR], kn, u);
-    u += fabsf(u) * 0x1p-20f;
-    if (FP8) {
-      u *= ks;
-      u += fabsf(u) * 0x1p-20f;
-    }
-    u = __fadd_rn(u, 0.f);  // -0 -> +0, as for scores
-    const bool vis = key < st->nvis[qi];
-    const bool skip = !vis || ordered_key(u) < st->thr[qi];
-    const uint32_t vb = __ballot_sync(kFullMask, vis);
-    const uint32_t bb = __ballot_sync(kFullMask, vis && skip);
-    const bool all_skip = __all_sync(kFullMask, skip);
-    if (lane == 0) {
-      screened += static_cast<unsigned long long>(__popc(vb));
-      bounded += static_cast<unsigned long long>(__popc(bb));
-      if (all_skip) skipped += static_cast<unsigned long long>(__popc(vb));
-    }
-    if (all_skip) {
-      s[qq] = -3.0e38f;
-      continue;
-    }
-    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                     make_float2(0.f, 0.f)};
-#pragma unroll
-    for (int h = 0; h < H; h += 4) {
-      const float4 wv = *reinterpret_cast<const float4*>(w + qq * H + h);
-      const float2 r01 = make_float2(relu2(r[qq * H + h + 0]),
-                                     relu2(r[qq * H + h + 1]));
-      const float2 r23 = make_float2(relu2(r[qq * H + h + 2]),
-                                     relu2(r[qq * H + h + 3]));
-      const int c = (h >> 2) & 1;
-      acc[2 * c] = __ffma2_rn(make_float2(wv.x, wv.y), r01, acc[2 * c]);
-      acc[2 * c + 1] = __ffma2_rn(make_float2(wv.z, wv.w), r23, acc[2 * c + 1]);
-    }
-    s[qq] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+  for (int h = 0; h < kPruneR; h += 4) {
+    const float4 wv = *reinterpret_cast<const float4*>(wt + h);
+    u0 = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(relu2(r[h]), relu2(r[h + 1])), u0);
+    u1 = __ffma2_rn(make_float2(wv.z, wv.w), make_float2(relu2(r[h + 2]), relu2(r[h + 3])), u1);
   }
+  float u = (u0.x + u0.y) + (u1.x + u1.y);
+  u = fmaf(wt[kPruneR], kn, u);
+  u += fabsf(u) * 0x1p-20f;
+  if (FP8) {
+    u *= ks;
+    u += fabsf(u) * 0x1p-20f;
+  }
+  return __fadd_rn(u, 0.f);  // -0 -> +0, as for scores
 }
 
 // ------------------------------------------------------------------------
@@ -613,7 +585,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const ScoreParams p) {
   using C = Cfg<H, D, FP8>;
-  constexpr int NQA = C::NQA;
   constexpr int NQW = C::NQW;
   constexpr int BN = C::BN;
   constexpr int QB = C::QB;
@@ -638,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->qempty, 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->accfull[a], 1);
-      mbar_init(&bars->accempty[a], 8);  // one arrival per warp of the two groups sharing it
+      mbar_init(&bars->accempty[a], 16);  // one arrival per epilogue warp
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -680,11 +651,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         first = false;
         mbar_arrive_expect_tx(&bars->qfull, C::Q_BYTES);
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-          for (int bx = 0; bx < C::NBOX; ++bx)
-            tma_load_2d(smem + C::OFF_Q + a * C::Q_ACC_BYTES + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS,
-                        (b * QB + a * NQA) * H, &bars->qfull);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_2d(smem + C::OFF_Q + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS, b * QB * H, &bars->qfull);
         for (int j = 0; j < nt; ++j) {
           ok = mbar_wait(&bars->kempty[stage], kph ^ 1u, abort_flag, kWaitLimitNs);
           if (!ok) break;
@@ -712,6 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t kph = 0, qf_ph = 0;
       uint32_t ae_ph[2] = {0u, 0u};
+      uint32_t tcount = 0;  // tiles issued so far; tile n goes to accumulator n & 1
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
@@ -726,26 +695,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t kst = k_base + stage * C::K_STAGE_BYTES;
-#pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            ok = mbar_wait(&bars->accempty[a], ae_ph[a] ^ 1u, abort_flag, kWaitLimitNs);
-            ae_ph[a] ^= 1u;
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t qa = q_base + a * C::Q_ACC_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < C::KSTEPS; ++kk) {
-              const uint64_t adesc = sw128_desc(kst + (kk >> 2) * (kBM * 128) + (kk & 3) * 32);
-              const uint64_t bdesc = sw128_desc(qa + (kk >> 2) * (BN * 128) + (kk & 3) * 32);
-              if constexpr (FP8)
-                tc_mma_e4m3(tmem_base + a * BN, adesc, bdesc, C::IDESC, kk > 0 ? 1u : 0u);
-              else
-                tc_mma_bf16(tmem_base + a * BN, adesc, bdesc, C::IDESC, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(&bars->accfull[a]);
-          }
+          const int a = static_cast<int>(tcount & 1u);
+          ok = mbar_wait(&bars->accempty[a], ae_ph[a] ^ 1u, abort_flag, kWaitLimitNs);
+          ae_ph[a] ^= 1u;
           if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint64_t adesc = sw128_desc(kst + (kk >> 2) * (kBM * 128) + (kk & 3) * 32);
+            const uint64_t bdesc = sw128_desc(q_base + (kk >> 2) * (BN * 128) + (kk & 3) * 32);
+            if constexpr (FP8)
+              tc_mma_e4m3(tmem_base + a * BN, adesc, bdesc, C::IDESC, kk > 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(tmem_base + a * BN, adesc, bdesc, C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars->accfull[a]);
           tc_commit(&bars->kempty[stage]);
+          ++tcount;
           if (++stage == STAGES) {
             stage = 0;
             kph ^= 1u;
@@ -773,17 +739,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     // ------------------------------------------------------ epilogue warpgroups
     const int eg = (warp - 4) >> 2;    // epilogue group 0..3
-    const int acc = eg >> 1;           // the accumulator it drains
-    const int half = eg & 1;           // which half of that accumulator's queries
     const int wq = warp & 3;           // TMEM lane quarter accessible to this warp
     const int etid = wq * 32 + lane;   // key row within the tile == order within the group
     const int bar_id = 1 + eg;
     WgState<NQW>* st = states + eg;
-    float* wsm = wsm_base + eg * (BN / 2);
+    float* wsm = wsm_base + eg * C::CW;
     uint32_t* hist = hist_base + eg * kHistBins;
-    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) +
-                           static_cast<uint32_t>(acc * BN + half * (BN / 2));
-    uint32_t af_ph = 0u;
+    // the group's columns eg*CW .. eg*CW+CW-1 of either accumulator hold its
+    // NQW queries (all H heads of each)
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(eg * C::CW);
+    uint32_t af_bits = 0u;  // phase parity of accumulator a's full barrier in bit a
+    uint32_t tcount = 0;    // tiles drained so far; tile n sits in accumulator n & 1
     int par = 0;
     bool failed = false;
     unsigned long long n_screened = 0ull, n_bounded = 0ull, n_skipped = 0ull;  // pruning counters (lane 0)
@@ -791,11 +757,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
       if (b < 0) break;
       const int nt = tiles_of_block<QB>(p, b);
-      const int64_t tq0 = static_cast<int64_t>(b) * QB + acc * NQA + half * NQW;
+      const int64_t tq0 = static_cast<int64_t>(b) * QB + eg * NQW;
       uint2* cand = p.cand + (static_cast<size_t>(blockIdx.x) * kEpiGroups + eg) * NQW * static_cast<size_t>(p.cap);
 
       named_bar(bar_id, kBM);  // the previous block is completely done with the state
-      for (int i = etid; i < BN / 2; i += kBM) {
+      for (int i = etid; i < C::CW; i += kBM) {
         const int64_t t = tq0 + i / H;
         float v = 0.f;
         if (t < p.S) {
@@ -826,13 +792,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per-tile path carries none of their code.
       int j = 0;
       while (true) {
+        // the group's head weights, in registers for the whole tile loop when
+        // they fit (reloaded after a cut, which needs the registers)
+        float wr[C::WREG ? C::CW - C::WSM_COLS : 4];
+        if constexpr (C::WREG) {
+#pragma unroll
+          for (int i = 0; i < C::CW - C::WSM_COLS; i += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(wsm + C::WSM_COLS + i);
+            wr[i] = v.x;
+            wr[i + 1] = v.y;
+            wr[i + 2] = v.z;
+            wr[i + 3] = v.w;
+          }
+        }
+        auto wget = [&](int col) -> float2 {
+          if (col < C::WSM_COLS) return *reinterpret_cast<const float2*>(wsm + col);
+          return make_float2(wr[col - C::WSM_COLS], wr[col - C::WSM_COLS + 1]);
+        };
+        // per-query state that only the selection steps change, in registers
+        // for the tile loop: candidates held, threshold, visible keys
+        int held[NQW];
+        uint32_t thr_r[NQW];
+        int32_t nvis_r[NQW];
+#pragma unroll
+        for (int qi = 0; qi < NQW; ++qi) {
+          held[qi] = st->cnt[par][qi];
+          thr_r[qi] = st->thr[qi];
+          nvis_r[qi] = st->nvis[qi];
+        }
         bool any_full = false;
         for (; j < nt; ++j) {
+          const int a = static_cast<int>(tcount & 1u);
+          ++tcount;
           // every lane polls (no divergent branch around the wait); the phase
           // is complete for all once any lane has seen it complete
-          bool ok = mbar_wait(&bars->accfull[acc], af_ph, abort_flag, kWaitLimitNs);
+          bool ok = mbar_wait(&bars->accfull[a], (af_bits >> a) & 1u, abort_flag, kWaitLimitNs);
           ok = __any_sync(kFullMask, ok);
-          af_ph ^= 1u;
+          af_bits ^= 1u << a;
           float s[NQW];
 #pragma unroll
           for (int qi = 0; qi < NQW; ++qi) s[qi] = 0.f;
@@ -842,27 +838,70 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (PRUNE) kn = key < p.n_keys ? p.knorm[key] : 0.f;
           if (ok) {
             tc_fence_after();
-            uint32_t ra[64];
+            const uint32_t tb = tbase + static_cast<uint32_t>(a * BN);
+            float2 acc[NQW][C::CHAINS];
 #pragma unroll
-            for (int c = 0; c < C::CHUNKS_W; ++c) {
-              tmem_ld_x64(tbase + c * 64, ra);
-              tmem_wait_ld(ra);
-              if (c + 1 == C::CHUNKS_W) {
-                // everything this warp needs from TMEM is in registers: hand the
-                // accumulator back before the last chunk's arithmetic
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->accempty[acc]);
-              }
-              bool pruned_path = false;
-              if constexpr (PRUNE && H >= 2 * kPruneR) {  // the host rejects pruning for fewer heads
-                {
-                  score_chunk_pruned<H, C::QPC, FP8, NQW>(ra, wsm + c * 64, s + c * C::QPC, st, c * C::QPC, key,
-                                                         ks, kn, lane, n_screened, n_bounded, n_skipped);
-                  pruned_path = true;
+            for (int qi = 0; qi < NQW; ++qi)
+#pragma unroll
+              for (int c = 0; c < C::CHAINS; ++c) acc[qi][c] = make_float2(0.f, 0.f);
+            if constexpr (PRUNE && H >= 2 * kPruneR) {  // the host rejects pruning for fewer heads
+              // per query: bound from its first 16 heads; the rest of its
+              // columns are read only if some key of the warp may pass
+              bool skip[NQW];
+#pragma unroll
+              for (int qi = 0; qi < NQW; ++qi) {
+                constexpr int CPQ = H / 16;  // chunks per query
+                uint32_t ra[16];
+                tmem_ld_x16(tb + qi * H, ra);
+                tmem_wait_ld(ra);
+                const float u = prune_bound<FP8>(ra, st->pq[qi], ks, kn);
+                const bool vis = key < st->nvis[qi];
+                const bool sk = !vis || ordered_key(u) < st->thr[qi];
+                const uint32_t vb = __ballot_sync(kFullMask, vis);
+                const uint32_t bb = __ballot_sync(kFullMask, vis && sk);
+                skip[qi] = __all_sync(kFullMask, sk);
+                if (lane == 0) {
+                  n_screened += static_cast<unsigned long long>(__popc(vb));
+                  n_bounded += static_cast<unsigned long long>(__popc(bb));
+                  if (skip[qi]) n_skipped += static_cast<unsigned long long>(__popc(vb));
+                }
+                if (skip[qi]) continue;
+                chunk_fma<H, NQW, C::CHAINS>(ra, qi * H, wget, acc);
+#pragma unroll
+                for (int c = 1; c < CPQ; ++c) {
+                  tmem_ld_x16(tb + qi * H + c * 16, ra);
+                  tmem_wait_ld(ra);
+                  chunk_fma<H, NQW, C::CHAINS>(ra, qi * H + c * 16, wget, acc);
                 }
               }
-              if (!pruned_path) score_chunk<H, C::QPC>(ra, wsm + c * 64, s + c * C::QPC);
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->accempty[a]);
+#pragma unroll
+              for (int qi = 0; qi < NQW; ++qi) s[qi] = skip[qi] ? -3.0e38f : chain_total<C::CHAINS>(acc[qi]);
+            } else {
+              // two chunk buffers: chunk c + 1 is on its way from TMEM while
+              // chunk c is summed
+              uint32_t ra[2][16];
+              tmem_ld_x16(tb, ra[0]);
+              tmem_wait_ld(ra[0]);
+#pragma unroll
+              for (int c = 0; c < C::NCH; ++c) {
+                if (c + 1 < C::NCH) tmem_ld_x16(tb + (c + 1) * 16, ra[(c + 1) & 1]);
+                chunk_fma<H, NQW, C::CHAINS>(ra[c & 1], c * 16, wget, acc);
+                if (c + 1 < C::NCH) {
+                  tmem_wait_ld(ra[(c + 1) & 1]);
+                  if (c + 2 == C::NCH) {
+                    // everything this warp needs from TMEM is in registers:
+                    // hand the accumulator back before the last chunk's sums
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->accempty[a]);
+                  }
+                }
+              }
+#pragma unroll
+              for (int qi = 0; qi < NQW; ++qi) s[qi] = chain_total<C::CHAINS>(acc[qi]);
             }
           }
           if constexpr (FP8) {
@@ -874,7 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int qi = 0; qi < NQW; ++qi) {
             okeys[qi] = ordered_key(__fadd_rn(s[qi], 0.f));
-            const bool pass = ok && key < st->nvis[qi] && okeys[qi] >= st->thr[qi];
+            const bool pass = ok && key < nvis_r[qi] && okeys[qi] >= thr_r[qi];
             bals[qi] = __ballot_sync(kFullMask, pass);
             if (lane == 0) reinterpret_cast<int32_t*>(&st->wc[par][qi])[wq] = __popc(bals[qi]);
           }
@@ -883,34 +922,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           // ordered append: position = held + earlier warps + earlier lanes.  No
-          // barrier follows: every thread knows the new counts, and the state read
-          // here is double-buffered by tile parity.
-          const int np = par ^ 1;
-          int newcnt[NQW];
+          // barrier follows: every thread knows the new counts, and the per-warp
+          // counts read here are double-buffered by tile parity.
           const uint32_t lt_mask = (1u << lane) - 1u;
 #pragma unroll
           for (int qi = 0; qi < NQW; ++qi) {
             const uint32_t bal = bals[qi];
-            const int held = st->cnt[par][qi];
             const int4 wc = st->wc[par][qi];
             const int tot = wc.x + wc.y + wc.z + wc.w;
             const int prior = (wq > 0 ? wc.x : 0) + (wq > 1 ? wc.y : 0) + (wq > 2 ? wc.z : 0);
             if ((bal >> lane) & 1u) {
-              const int pos = held + prior + __popc(bal & lt_mask);
+              const int pos = held[qi] + prior + __popc(bal & lt_mask);
               cand[qi * static_cast<size_t>(p.cap) + pos] = make_uint2(okeys[qi], static_cast<uint32_t>(key));
             }
-            newcnt[qi] = held + tot;
-            if (etid == qi) st->cnt[np][qi] = held + tot;
+            held[qi] += tot;
           }
-          par = np;
+          par ^= 1;
 #pragma unroll
-          for (int qi = 0; qi < NQW; ++qi) any_full |= newcnt[qi] > p.cap - kBM;
+          for (int qi = 0; qi < NQW; ++qi) any_full |= held[qi] > p.cap - kBM;
           if (any_full) {
             ++j;
             break;
           }
         }
         if (failed) break;
+#pragma unroll
+        for (int qi = 0; qi < NQW; ++qi)
+          if (etid == qi) st->cnt[par][qi] = held[qi];
         // no buffer is full: the block's tiles are done and the final top-K of
         // each query is written; otherwise the full buffers are cut back
         const bool fin = !any_full;
