@@ -97,8 +97,12 @@ struct Cfg {
   static constexpr int CW = BN / 4;                      // columns (query, head) per epilogue warpgroup
   static constexpr int NQW = CW / H;                     // queries per epilogue warpgroup
   static constexpr int NCH = CW / 16;                    // 16-column TMEM loads per warpgroup and tile
-  static constexpr bool WREG = NQW <= 2;                 // head weights held in registers
-  static constexpr int WSM_COLS = WREG ? 16 : CW;         // columns whose weights stay in shared memory
+  // Columns whose head weights are read from shared memory each tile; the
+  // rest stay in registers for the whole block.  Measured per variant: the
+  // bf16 one-query groups run fastest with every weight in registers, the FP8
+  // and two-query groups with 16 in registers (register pressure elsewhere).
+  static constexpr bool WREG = NQW <= 2;
+  static constexpr int WSM_COLS = !WREG ? CW : ((!FP8 && NQW == 1) ? 0 : 48);
   static constexpr int CHAINS = NQW == 1 ? 4 : 2;        // packed partial sums per query
   static constexpr int Q_ACC_BYTES = BN * ROW_BYTES;
   static constexpr int Q_BYTES = Q_ACC_BYTES;
@@ -589,6 +593,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int BN = C::BN;
   constexpr int QB = C::QB;
   constexpr int STAGES = C::STAGES;
+  // the pruning screen needs registers of its own: keep 48 columns' weights in
+  // shared memory there
+  constexpr int kWsm = (PRUNE && C::WREG) ? 48 : C::WSM_COLS;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -794,11 +801,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (true) {
         // the group's head weights, in registers for the whole tile loop when
         // they fit (reloaded after a cut, which needs the registers)
-        float wr[C::WREG ? C::CW - C::WSM_COLS : 4];
-        if constexpr (C::WREG) {
+        float wr[C::CW > kWsm ? C::CW - kWsm : 4];
+        if constexpr (C::CW > kWsm) {
 #pragma unroll
-          for (int i = 0; i < C::CW - C::WSM_COLS; i += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(wsm + C::WSM_COLS + i);
+          for (int i = 0; i < C::CW - kWsm; i += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(wsm + kWsm + i);
             wr[i] = v.x;
             wr[i + 1] = v.y;
             wr[i + 2] = v.z;
@@ -806,8 +813,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         auto wget = [&](int col) -> float2 {
-          if (col < C::WSM_COLS) return *reinterpret_cast<const float2*>(wsm + col);
-          return make_float2(wr[col - C::WSM_COLS], wr[col - C::WSM_COLS + 1]);
+          if (col < kWsm) return *reinterpret_cast<const float2*>(wsm + col);
+          return make_float2(wr[col - kWsm], wr[col - kWsm + 1]);
         };
         // per-query state that only the selection steps change, in registers
         // for the tile loop: candidates held, threshold, visible keys
