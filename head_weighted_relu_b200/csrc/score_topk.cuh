@@ -103,7 +103,7 @@ struct Cfg {
   // and two-query groups with 16 in registers (register pressure elsewhere).
   static constexpr bool WREG = NQW <= 2;
   static constexpr int WSM_COLS = !WREG ? CW : ((!FP8 && NQW == 1) ? 0 : 48);
-  static constexpr int CHAINS = NQW == 1 ? 4 : 2;        // packed partial sums per query
+  static constexpr int CHAINS = 2;                       // packed partial sums per query (fewest registers)
   static constexpr int Q_ACC_BYTES = BN * ROW_BYTES;
   static constexpr int Q_BYTES = Q_ACC_BYTES;
   static constexpr int K_STAGE_BYTES = kBM * ROW_BYTES;
@@ -151,12 +151,13 @@ __device__ __forceinline__ int tiles_of_block(const ScoreParams& p, int b) {
   return (n + kBM - 1) / kBM;
 }
 
-// 2 * max(x, 0) for the accumulator bits of x, computed as x + |x| on the FMA
-// pipe (exact: 2x for x >= 0, +0 otherwise).  The head weights are staged
-// halved (also exact), so w/2 * (x + |x|) rounds exactly like w * max(x, 0).
-__device__ __forceinline__ float relu2(uint32_t bits) {
-  const float x = __uint_as_float(bits);
-  return x + fabsf(x);
+// 2 * max(x, 0) for two accumulator columns, computed as x + |x| with one
+// packed add (exact: 2x for x >= 0, +0 otherwise).  The head weights are
+// staged halved (also exact), so w/2 * (x + |x|) rounds exactly like
+// w * max(x, 0).
+__device__ __forceinline__ float2 relu2x2(uint32_t b0, uint32_t b1) {
+  const float2 x = make_float2(__uint_as_float(b0), __uint_as_float(b1));
+  return __fadd2_rn(x, make_float2(fabsf(x.x), fabsf(x.y)));
 }
 
 // Adds one 16-column TMEM chunk of the group's columns into the packed partial
@@ -173,7 +174,7 @@ __device__ __forceinline__ void chunk_fma(const uint32_t (&r)[16], int col0, WGe
     const int col = col0 + k;
     const int qi = col / H;
     const int ch = ((col % H) >> 1) % CHAINS;
-    acc[qi][ch] = __ffma2_rn(wget(col), make_float2(relu2(r[k]), relu2(r[k + 1])), acc[qi][ch]);
+    acc[qi][ch] = __ffma2_rn(wget(col), relu2x2(r[k], r[k + 1]), acc[qi][ch]);
   }
 }
 
@@ -195,8 +196,8 @@ __device__ __forceinline__ float prune_bound(const uint32_t (&r)[16], const floa
 #pragma unroll
   for (int h = 0; h < kPruneR; h += 4) {
     const float4 wv = *reinterpret_cast<const float4*>(wt + h);
-    u0 = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(relu2(r[h]), relu2(r[h + 1])), u0);
-    u1 = __ffma2_rn(make_float2(wv.z, wv.w), make_float2(relu2(r[h + 2]), relu2(r[h + 3])), u1);
+    u0 = __ffma2_rn(make_float2(wv.x, wv.y), relu2x2(r[h], r[h + 1]), u0);
+    u1 = __ffma2_rn(make_float2(wv.z, wv.w), relu2x2(r[h + 2], r[h + 3]), u1);
   }
   float u = (u0.x + u0.y) + (u1.x + u1.y);
   u = fmaf(wt[kPruneR], kn, u);

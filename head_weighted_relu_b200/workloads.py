@@ -46,6 +46,7 @@ class Workload:
     q_pos0: int = 0
     seed: int = 0
     values: str = "gauss"        # "gauss", "int", or "corr" (correlated heads, w >= 0)
+    pair_overlap: bool = False   # the step also counts shared indices of adjacent query pairs
 
     def problem(self) -> dict:
         return dict(S=self.S, T=self.T, H=self.H, D=self.D, K=self.K,
@@ -70,7 +71,7 @@ WORKLOADS = {
                                  seed=3),
     "long_1m_fp8": Workload("long_1m_fp8", S=16384, T=1048576, H=64, D=128,
                             K=2048, dtype="fp8", q_pos0=1048576 - 16384,
-                            seed=4),
+                            seed=4, pair_overlap=True),
 }
 
 
