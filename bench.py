@@ -240,6 +240,26 @@ def main():
     value = pairs * world / (ms_step * 1e-3) / 1e9
     peak_mem = torch.cuda.max_memory_allocated(dev) / 1e9
 
+    # the q-cluster preprocessing of the same pairs (shared / left-only /
+    # right-only regions), timed on its own on this step's index rows
+    regions = None
+    if shared is not None:
+        width = bufs[0].shape[1]
+        outs = [torch.empty((wl.S // 2, width), dtype=torch.int32, device=dev) for _ in range(3)]
+        cnt = torch.empty((wl.S // 2, 3), dtype=torch.int32, device=dev)
+        for _ in range(3):
+            I.indexer_pair_regions(bufs[0], bufs[1], wl.S, width, *outs, cnt, stream)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(10):
+            I.indexer_pair_regions(bufs[0], bufs[1], wl.S, width, *outs, cnt, stream)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        r_ms = r0.elapsed_time(r1) / 10
+        r_bytes = (bufs[0].numel() + bufs[1].numel() + 3 * outs[0].numel() + cnt.numel()) * 4
+        regions = {"ms_per_call": r_ms, "bytes_per_call": r_bytes, "gb_s": r_bytes / (r_ms * 1e-3) / 1e9}
+        del outs, cnt
+
     pk = _peaks()
     tensor_peak = pk["bf16"] * (2.0 if wl.dtype == "fp8" else 1.0)
     kern_ms = statistics.mean(per)
@@ -320,6 +340,7 @@ def main():
             "clocks": clk.summary(),
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
+            "pair_regions": regions,
             "device_status": status,
             "cpu_baseline": base,
         }

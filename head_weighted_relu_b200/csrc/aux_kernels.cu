@@ -1,10 +1,13 @@
-// aux_kernels.cu -- the two small steps around the scoring kernel:
+// aux_kernels.cu -- the small steps around the scoring kernel:
 //   * pool formation for pooled indexing ("Module 06 — DSA & KPool:
 //     Selective Retrieval", §2: a channel-wise weighted representation of each
 //     complete pool of 4 tokens), and
 //   * exact shared-index counts of adjacent query pairs ("Adjacent-Query
 //     KV-Index Overlap in 256K DSA Training", §1 pairs (q0,q1),(q2,q3),...;
-//     §3 exact intersections by batched binary search).
+//     §3 exact intersections by batched binary search), and
+//   * the shared / left-only / right-only index regions of those pairs (same
+//     page, §6.1 and §6.4: q-cluster preprocessing into fixed-capacity
+//     buffers with device-side counts).
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -111,6 +114,85 @@ __global__ void pair_overlap_kernel(const int32_t* __restrict__ idx, const int32
     count = warp_sum_i32(count);
     if (lane == 0) out[pr] = count;
   }
+}
+
+// True when the strictly ascending row b[0, lb) holds x (binary search).
+__device__ __forceinline__ bool row_holds(const int32_t* __restrict__ b, int lb, int32_t x) {
+  int lo = 0, hi = lb;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (b[mid] < x)
+      lo = mid + 1;
+    else
+      hi = mid;
+  }
+  return lo < lb && b[lo] == x;
+}
+
+// One warp per pair.  The rows are ascending, so taking a row's entries in
+// order keeps every region ascending: the warp tests 32 consecutive entries
+// against the other row and writes each region's members at the region's
+// running length plus their ballot rank.
+__global__ void pair_regions_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ len,
+                                    int64_t n_pairs, int width, int32_t* __restrict__ shared,
+                                    int32_t* __restrict__ left, int32_t* __restrict__ right,
+                                    int32_t* __restrict__ counts) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t pr = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); pr < n_pairs;
+       pr += warps) {
+    const int32_t* a = idx + (2 * pr) * width;
+    const int32_t* b = idx + (2 * pr + 1) * width;
+    const int la = min(max(len[2 * pr], 0), width);
+    const int lb = min(max(len[2 * pr + 1], 0), width);
+    int32_t* so = shared + pr * width;
+    int32_t* lo = left + pr * width;
+    int32_t* ro = right + pr * width;
+    int ns = 0, nl = 0, nr = 0;
+    for (int base = 0; base < la; base += 32) {
+      const int i = base + lane;
+      const bool in = i < la;
+      const int32_t x = in ? a[i] : 0;
+      const bool both = in && row_holds(b, lb, x);
+      const uint32_t bs = __ballot_sync(kFullMask, both);
+      const uint32_t bl = __ballot_sync(kFullMask, in && !both);
+      if (both) so[ns + __popc(bs & lt)] = x;
+      if (in && !both) lo[nl + __popc(bl & lt)] = x;
+      ns += __popc(bs);
+      nl += __popc(bl);
+    }
+    for (int base = 0; base < lb; base += 32) {
+      const int i = base + lane;
+      const bool only = i < lb && !row_holds(a, la, b[i]);
+      const uint32_t br = __ballot_sync(kFullMask, only);
+      if (only) ro[nr + __popc(br & lt)] = b[i];
+      nr += __popc(br);
+    }
+    for (int i = ns + lane; i < width; i += 32) so[i] = -1;
+    for (int i = nl + lane; i < width; i += 32) lo[i] = -1;
+    for (int i = nr + lane; i < width; i += 32) ro[i] = -1;
+    if (lane == 0) {
+      counts[3 * pr] = ns;
+      counts[3 * pr + 1] = nl;
+      counts[3 * pr + 2] = nr;
+    }
+  }
+}
+
+cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
+                                int32_t* shared, int32_t* left, int32_t* right, int32_t* counts,
+                                cudaStream_t stream) {
+  if (n_pairs == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int threads = 256;  // 8 pairs per block
+  int64_t blocks = (n_pairs + 7) / 8;
+  if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+  pair_regions_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, len, n_pairs, width, shared,
+                                                                            left, right, counts);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_pair_overlap(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,

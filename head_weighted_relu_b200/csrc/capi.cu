@@ -280,6 +280,18 @@ indexer_status indexer_pair_overlap(const int32_t* idx, const int32_t* len, int6
   return INDEXER_OK;
 }
 
+indexer_status indexer_pair_regions(const int32_t* idx, const int32_t* len, int64_t S, int32_t width,
+                                    int32_t* out_shared, int32_t* out_left, int32_t* out_right,
+                                    int32_t* out_counts, void* stream) {
+  if (S < 0 || width < 0) return INDEXER_EINVAL;
+  if (S / 2 == 0) return INDEXER_OK;
+  if (!idx || !len || !out_shared || !out_left || !out_right || !out_counts) return INDEXER_EINVAL;
+  if (launch_pair_regions(idx, len, S / 2, width, out_shared, out_left, out_right, out_counts,
+                          static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return INDEXER_ECUDA;
+  return INDEXER_OK;
+}
+
 indexer_status indexer_read_prune_counters(void* workspace, uint64_t* counts, void* stream) {
   if (!workspace || !counts) return INDEXER_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

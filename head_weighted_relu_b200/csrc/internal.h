@@ -73,6 +73,9 @@ cudaError_t launch_pool_keys(const void* k, int64_t n_pools, int D, const void* 
 cudaError_t launch_prune_setup(const void* q, const float* w, const float* q_scale, bool fp8, int64_t S, int H,
                                int D, const void* keys, int64_t n_keys, float* pq, float* knorm,
                                cudaStream_t stream);
+cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
+                                int32_t* shared, int32_t* left, int32_t* right, int32_t* counts,
+                                cudaStream_t stream);
 cudaError_t launch_pair_overlap(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
                                 int32_t* out, cudaStream_t stream);
 

@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
 # every symbol include/hwr_indexer.h declares
 EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_topk_noalloc",
            "indexer_pool_keys",
-           "indexer_pair_overlap", "indexer_read_status", "indexer_read_prune_counters",
+           "indexer_pair_overlap", "indexer_pair_regions", "indexer_read_status", "indexer_read_prune_counters",
            "indexer_status_string",
            "indexer_abi_version")
 
@@ -64,6 +64,7 @@ def _load():
     lib.indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.indexer_pool_keys.argtypes = [vp, i64, i32, vp, i32, vp, vp]
     lib.indexer_pair_overlap.argtypes = [vp, vp, i64, i32, vp, vp]
+    lib.indexer_pair_regions.argtypes = [vp, vp, i64, i32, vp, vp, vp, vp, vp]
     lib.indexer_read_status.argtypes = [vp, ctypes.POINTER(i32), vp]
     lib.indexer_read_prune_counters.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), vp]
     lib.indexer_status_string.argtypes = [ctypes.c_int]
@@ -143,6 +144,12 @@ def indexer_pair_overlap(idx, lens, S, width, out_shared, stream=None):
         _ptr(idx), _ptr(lens), S, width, _ptr(out_shared), _stream(stream)))
 
 
+def indexer_pair_regions(idx, lens, S, width, out_shared, out_left, out_right, out_counts, stream=None):
+    _check("indexer_pair_regions", _lib.indexer_pair_regions(
+        _ptr(idx), _ptr(lens), S, width, _ptr(out_shared), _ptr(out_left), _ptr(out_right), _ptr(out_counts),
+        _stream(stream)))
+
+
 def indexer_read_status(workspace, stream=None) -> int:
     f = ctypes.c_int32()
     _check("indexer_read_status",
@@ -218,6 +225,16 @@ def pair_overlap(idx, lens, stream=None):
     out = torch.empty((S // 2,), dtype=torch.int32, device=idx.device)
     indexer_pair_overlap(idx.contiguous(), lens.contiguous(), S, width, out, stream)
     return out
+
+
+def pair_regions(idx, lens, stream=None):
+    """Shared, left-only and right-only KV indices of each adjacent query pair,
+    each [S/2, width] (ascending, -1 padded), and their lengths [S/2, 3]."""
+    S, width = idx.shape
+    outs = [torch.empty((S // 2, width), dtype=torch.int32, device=idx.device) for _ in range(3)]
+    counts = torch.empty((S // 2, 3), dtype=torch.int32, device=idx.device)
+    indexer_pair_regions(idx.contiguous(), lens.contiguous(), S, width, *outs, counts, stream)
+    return outs[0], outs[1], outs[2], counts
 
 
 def pool_keys(k, pool_coef, ratio, stream=None):

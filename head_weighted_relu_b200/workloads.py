@@ -138,6 +138,37 @@ def generate(wl: Workload, device="cpu") -> dict:
     return out
 
 
+def index_rows(S: int, width: int, universe: int, seed: int):
+    """Seeded rows shaped like the indexer's output, for the pair steps:
+    row r holds len[r] distinct ascending KV indices below `universe`, then -1
+    padding.  Lengths cover 0 and width; pair 1 has two identical rows, pair 2
+    two disjoint rows, and the other odd rows re-use about three quarters of
+    their partner's indices (the high-overlap regime the pair steps target).
+    Returns numpy int32 arrays idx [S, width] and len [S]."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    idx = np.full((S, width), -1, dtype=np.int32)
+    ln = np.zeros(S, dtype=np.int32)
+    for r in range(S):
+        n = int(rng.integers(0, width + 1)) if r > 5 else [0, width, width, width, width // 2, width // 2][r]
+        if r in (3,):
+            row = idx[2, : ln[2]]
+        elif r == 5:
+            taken = set(idx[4, : ln[4]].tolist())
+            free = np.array([v for v in range(universe) if v not in taken])
+            row = np.sort(rng.choice(free, size=min(n, free.size), replace=False))
+        elif r % 2 == 1 and ln[r - 1] > 0:
+            prev = idx[r - 1, : ln[r - 1]]
+            keep = prev[rng.random(prev.size) < 0.75]
+            extra = rng.choice(universe, size=max(n - keep.size, 0), replace=False)
+            row = np.unique(np.concatenate([keep, extra]))[:width]
+        else:
+            row = np.sort(rng.choice(universe, size=n, replace=False))
+        idx[r, : row.size] = row
+        ln[r] = row.size
+    return idx, ln
+
+
 def sample_rows(wl: Workload, n: int = 1024, seed: int = 12345) -> np.ndarray:
     """Seeded query rows for the oracle: the first 4 rows, rows whose global
     position is near K (K-2 .. K+1) and near the first pool boundaries, the

@@ -180,6 +180,25 @@ indexer_status indexer_pair_overlap(const int32_t* idx, const int32_t* len,
                                     int64_t S, int32_t width,
                                     int32_t* out_shared, void* stream);
 
+/* The three index regions of the same pairs, the preprocessing of a
+ * two-query cluster ("Adjacent-Query KV-Index Overlap in 256K DSA Training",
+ * §6.1: indices both queries select, and those only the left or only the
+ * right query selects; §6.4: fixed-capacity buffers with device-side counts,
+ * so a captured CUDA graph keeps its shapes):
+ *   shared[p] = A ∩ B,  left[p] = A \ B,  right[p] = B \ A,
+ *   A = idx[2p, :len[2p]],  B = idx[2p+1, :len[2p+1]],
+ * each in ascending KV order at the start of row p of its [S/2, width] int32
+ * buffer, padded with -1; out_counts[3p + r] is the length of region r
+ * (0 shared, 1 left, 2 right).  Valid prefixes must be strictly ascending (as
+ * indexer_topk writes them).  All buffers are caller-owned device memory;
+ * nothing is allocated and the host does not wait.  INDEXER_EINVAL for a
+ * negative S or width or a null pointer (when S >= 2). */
+indexer_status indexer_pair_regions(const int32_t* idx, const int32_t* len,
+                                    int64_t S, int32_t width,
+                                    int32_t* out_shared, int32_t* out_left,
+                                    int32_t* out_right, int32_t* out_counts,
+                                    void* stream);
+
 /* Synchronises `stream`, then reads the device status word that indexer_topk
  * keeps in `workspace` (0 = no fault).  Bit 0: a pipeline wait in the kernel
  * gave up after its time limit (the result is not valid); bit 1: a candidate

@@ -27,4 +27,5 @@ from .indexer_oracle import (  # noqa: F401
     topk_rows,
     decode_keys_for,
     pair_shared_counts,
+    pair_regions,
 )

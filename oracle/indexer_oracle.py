@@ -344,3 +344,33 @@ def pair_shared_counts(idx, lens) -> np.ndarray:
         both = np.sort(np.concatenate([a, b]), kind="stable")
         out[p] = int(np.count_nonzero(both[1:] == both[:-1]))
     return out
+
+
+def pair_regions(idx, lens, width: int):
+    """The three index regions of each non-overlapping adjacent query pair.
+
+    "Adjacent-Query KV-Index Overlap in 256K DSA Training", §6.1: a two-query
+    cluster splits its selection into the indices both queries select, those
+    only the left query (row 2p) selects, and those only the right query (row
+    2p+1) selects; §6.4: each region goes to a buffer of fixed capacity (the
+    row width), with its length as a device-side count.  Here the regions are
+    the set intersection and the two set differences of the valid prefixes,
+    each listed in ascending KV order and padded with -1.
+
+    Returns shared, left, right [S/2, width] int32 and counts [S/2, 3] int32
+    (shared, left-only, right-only).
+    """
+    idx = np.asarray(idx)
+    lens = np.asarray(lens)
+    n_pairs = idx.shape[0] // 2
+    regions = [np.full((n_pairs, width), -1, dtype=np.int32) for _ in range(3)]
+    counts = np.zeros((n_pairs, 3), dtype=np.int32)
+    for p in range(n_pairs):
+        a = set(int(v) for v in idx[2 * p, : lens[2 * p]])
+        b = set(int(v) for v in idx[2 * p + 1, : lens[2 * p + 1]])
+        for r, members in enumerate((a & b, a - b, b - a)):
+            ordered = sorted(members)
+            regions[r][p, : len(ordered)] = ordered
+            counts[p, r] = len(ordered)
+    return regions[0], regions[1], regions[2], counts
+

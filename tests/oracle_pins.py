@@ -387,6 +387,45 @@ def pin_pair_overlap(O):
     assert O.pair_shared_counts(idx2, ln2).tolist() == [1, 3, 5]
 
 
+def pin_pair_regions(O):
+    """Shared / left-only / right-only regions of a pair ("Adjacent-Query
+    KV-Index Overlap in 256K DSA Training", §6.1, §6.4): a hand example, then
+    properties on random rows -- shared + left rebuilds the left row, shared +
+    right the right row, the three regions are disjoint and ascending, and the
+    shared length equals the overlap count computed by the independent
+    sort-and-count method."""
+    idx = np.array([[1, 3, 5, 7, -1], [3, 4, 7, 9, 11]], np.int32)
+    sh, le, ri, c = O.pair_regions(idx, np.array([4, 5], np.int32), 5)
+    assert sh[0].tolist() == [3, 7, -1, -1, -1]
+    assert le[0].tolist() == [1, 5, -1, -1, -1]
+    assert ri[0].tolist() == [4, 9, 11, -1, -1]
+    assert c[0].tolist() == [2, 2, 3]
+    rng = np.random.default_rng(31)
+    S, W = 41, 24   # odd: the last row has no partner
+    idx = np.full((S, W), -1, dtype=np.int32)
+    ln = np.zeros(S, dtype=np.int32)
+    for r in range(S):
+        n = int(rng.integers(0, W + 1))
+        idx[r, :n] = np.sort(rng.choice(40, size=n, replace=False))
+        ln[r] = n
+    idx[2, : ln[3]] = idx[3, : ln[3]]   # one pair of identical rows
+    ln[2] = ln[3]
+    sh, le, ri, c = O.pair_regions(idx, ln, W)
+    assert sh.shape == (S // 2, W) and c.shape == (S // 2, 3)
+    assert np.array_equal(c[:, 0], O.pair_shared_counts(idx, ln))
+    for p in range(S // 2):
+        a = idx[2 * p, : ln[2 * p]].tolist()
+        b = idx[2 * p + 1, : ln[2 * p + 1]].tolist()
+        ns, nl, nr = c[p].tolist()
+        s_, l_, r_ = sh[p, :ns].tolist(), le[p, :nl].tolist(), ri[p, :nr].tolist()
+        assert sorted(s_ + l_) == a and sorted(s_ + r_) == b, p
+        assert not (set(s_) & set(l_)) and not (set(s_) & set(r_)) and not (set(l_) & set(r_)), p
+        for region in (s_, l_, r_):
+            assert region == sorted(region)
+        assert (sh[p, ns:] == -1).all() and (le[p, nl:] == -1).all() and (ri[p, nr:] == -1).all()
+    assert c[1, 1] == 0 and c[1, 2] == 0   # identical rows: nothing unique
+
+
 def pin_fp8_scales(O):
     """An FP8 value means code * row scale: doubling every key scale doubles
     every score and leaves the selection unchanged; a per-(query, head) scale
@@ -432,5 +471,6 @@ PINS = [
     pin_e4m3_decoder,
     pin_bf16_codec,
     pin_pair_overlap,
+    pin_pair_regions,
     pin_fp8_scales,
 ]

@@ -138,9 +138,8 @@ def test_deterministic_and_pair_overlap(cuda_ok):
                            y.nan_to_num(-7.0) if y.is_floating_point() else y)
     shared = I.pair_overlap(a[0], a[1])
     torch.cuda.synchronize()
-    ref = oracle.pair_shared_counts(a[0].cpu().numpy(), a[1].cpu().numpy())
-    assert np.array_equal(shared.cpu().numpy(), ref)
-    # rows 0..K-1 see their whole prefix: shared = length of the even row
+    # rows 0..K-1 see their whole prefix: shared = length of the even row (the
+    # oracle comparison of the pair steps is in test_gpu_pairs.py)
     assert shared[: wl.K // 2].cpu().tolist() == [2 * p + 1 for p in range(wl.K // 2)]
 
 

@@ -31,6 +31,9 @@ MUTATIONS = {
     "fp8_key_scale_ignored": ("return decode_e4m3(k) * np.asarray(k_scale, dtype=np.float64)[:, None]",
                               "return decode_e4m3(k)"),
     "tail_before_pools": ("pos = np.concatenate([pos, tail])", "pos = np.concatenate([tail, pos])"),
+    "regions_left_right_swapped": ("for r, members in enumerate((a & b, a - b, b - a)):",
+                                   "for r, members in enumerate((a & b, b - a, a - b)):"),
+    "regions_unsorted": ("            ordered = sorted(members)", "            ordered = sorted(members, reverse=True)"),
 }
 
 
