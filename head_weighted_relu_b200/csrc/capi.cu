@@ -70,6 +70,11 @@ struct Plan {
   size_t kn_bytes;   // key norms (pruning only)
   bool prune;
   size_t cand_bytes;
+  int32_t splits;          // key-range splits per query block (1: none)
+  size_t split_bytes;      // per-split top-K lists
+  int64_t gather_stride;   // entries per query of the merge's gathered list (a multiple of 128)
+  size_t gather_bytes;
+  size_t split_cnt_bytes;  // per-split list lengths
   size_t ws_bytes;
 };
 
@@ -105,13 +110,40 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
   pl->cap = candidate_capacity(pl->ksel);
   pl->grid = 0;
   pl->cand_bytes = 0;
+  pl->splits = 1;
+  pl->split_bytes = 0;
+  pl->gather_stride = 0;
+  pl->gather_bytes = 0;
+  pl->split_cnt_bytes = 0;
   if (need_device) {
     DeviceInfo di;
     const indexer_status st = device_info(&di);
     if (st != INDEXER_OK) return st;
-    pl->grid = static_cast<int32_t>(nb < di.sms ? nb : di.sms);
+    // Fewer query blocks than half the SMs (decode-like shapes): cut each
+    // block's key tiles into consecutive ranges of at least 16 tiles, one CTA
+    // each, so that every SM has work; a merge step joins the ranges.
+    if (nb > 0 && nb * 2 <= di.sms) {
+      const int64_t g_last = p->q_pos0 + p->S - 1;
+      int64_t nvis = pl->ranged ? (g_last + 1) / ratio : g_last + 1;
+      if (nvis > pl->n_keys) nvis = pl->n_keys;
+      int64_t s = di.sms / nb;
+      const int64_t by_tiles = (nvis + 127) / 128 / 16;
+      if (s > by_tiles) s = by_tiles;
+      if (s > kMaxSplits) s = kMaxSplits;
+      if (s >= 2) pl->splits = static_cast<int32_t>(s);
+    }
+    const int64_t items = nb * pl->splits;
+    pl->grid = static_cast<int32_t>(items < di.sms ? items : di.sms);
     pl->cand_bytes = static_cast<size_t>(pl->grid) * pl->var.groups * pl->var.queries_per_wg *
                      static_cast<size_t>(pl->cap) * sizeof(uint2);
+    if (pl->splits > 1) {
+      pl->split_bytes = align256(static_cast<size_t>(p->S) * pl->splits * pl->ksel * sizeof(uint2));
+      // the selection reads entries in pairs: a padded stride keeps those reads
+      // inside the query's own region
+      pl->gather_stride = (static_cast<int64_t>(pl->splits) * pl->ksel + 127) / 128 * 128;
+      pl->gather_bytes = align256(static_cast<size_t>(p->S) * pl->gather_stride * sizeof(uint2));
+      pl->split_cnt_bytes = align256(static_cast<size_t>(p->S) * pl->splits * sizeof(int32_t));
+    }
   }
   pl->kp_bytes = p->visibility == INDEXER_VIS_POOLED
                      ? align256(static_cast<size_t>(pl->n_keys) * p->D * 2)
@@ -120,7 +152,8 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
   if (pl->prune && (p->H < 2 * kPruneR || p->D % 32 != 0 || p->D > 128)) return INDEXER_EUNSUPPORTED;
   pl->pq_bytes = pl->prune ? align256(static_cast<size_t>(p->S) * (kPruneR + 2) * sizeof(float)) : 0;
   pl->kn_bytes = pl->prune ? align256(static_cast<size_t>(pl->n_keys) * sizeof(float)) : 0;
-  pl->ws_bytes = kStatusBytes + pl->kp_bytes + pl->pq_bytes + pl->kn_bytes + align256(pl->cand_bytes);
+  pl->ws_bytes = kStatusBytes + pl->kp_bytes + pl->pq_bytes + pl->kn_bytes + align256(pl->cand_bytes) +
+                 pl->split_bytes + pl->gather_bytes + pl->split_cnt_bytes;
   return INDEXER_OK;
 }
 
@@ -206,6 +239,10 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   float* pq = reinterpret_cast<float*>(ws + kStatusBytes + pl.kp_bytes);
   float* knorm = reinterpret_cast<float*>(ws + kStatusBytes + pl.kp_bytes + pl.pq_bytes);
   uint2* cand = reinterpret_cast<uint2*>(ws + kStatusBytes + pl.kp_bytes + pl.pq_bytes + pl.kn_bytes);
+  uint8_t* split_base = reinterpret_cast<uint8_t*>(cand) + align256(pl.cand_bytes);
+  uint2* split_buf = reinterpret_cast<uint2*>(split_base);
+  uint2* split_gather = reinterpret_cast<uint2*>(split_base + pl.split_bytes);
+  int32_t* split_cnt = reinterpret_cast<int32_t*>(split_base + pl.split_bytes + pl.gather_bytes);
   // status word and the three pruning counters (bytes 0, 8, 16, 24) start at zero
   if (cudaMemsetAsync(status, 0, 32, stream) != cudaSuccess) return INDEXER_ECUDA;
   if (p->S == 0) return INDEXER_OK;
@@ -246,16 +283,22 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   sp.pq = pq;
   sp.knorm = knorm;
   sp.counters = reinterpret_cast<unsigned long long*>(ws + 8);
+  sp.splits = pl.splits;
+  sp.split_buf = split_buf;
+  sp.split_cnt = split_cnt;
   if (pl.prune && launch_prune_setup(q, w, q_scale, fp8, p->S, p->H, p->D, keys, pl.n_keys, pq, knorm,
                                      stream) != cudaSuccess)
     return INDEXER_ECUDA;
 
-  if (cudaFuncSetAttribute(pl.var.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.var.smem_bytes) !=
-      cudaSuccess)
+  const void* fn = pl.splits > 1 ? pl.var.fn_split : pl.var.fn;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.var.smem_bytes) != cudaSuccess)
     return INDEXER_ECUDA;
   void* args[] = {&tm_q, &tm_k, &sp};
-  if (cudaLaunchKernel(pl.var.fn, dim3(pl.grid), dim3(pl.var.threads), args, pl.var.smem_bytes, stream) !=
-      cudaSuccess)
+  if (cudaLaunchKernel(fn, dim3(pl.grid), dim3(pl.var.threads), args, pl.var.smem_bytes, stream) != cudaSuccess)
+    return INDEXER_ECUDA;
+  if (pl.splits > 1 &&
+      launch_merge_splits(p->S, p->q_pos0, pl.splits, pl.ksel, pl.width, pl.out_ratio, split_buf, split_cnt,
+                          split_gather, pl.gather_stride, out_idx, out_len, out_score, stream) != cudaSuccess)
     return INDEXER_ECUDA;
   return INDEXER_OK;
 }

@@ -39,11 +39,15 @@ struct ScoreParams {
   const float* pq;             // [S][kPruneR + 2]: folded weights wt[0..r), Ceff, sum |w||q|
   const float* knorm;          // [n_keys]: |k_i| in the kernel's domain, rounded up
   unsigned long long* counters;  // [3]: pairs screened, bounded below the threshold, skipped
+  int32_t splits;        // key-range splits per query block (1: each block is one work item)
+  uint2* split_buf;      // splits > 1: [S][splits][ksel] top-K of each split, in key order
+  int32_t* split_cnt;    // splits > 1: [S][splits] entries of each split
 };
 
 // Per-variant launch facts, filled by the kernel's translation unit.
 struct ScoreVariant {
   const void* fn;         // kernel function
+  const void* fn_split;   // the same with key ranges split across CTAs (ScoreParams::splits > 1)
   int queries_per_block;  // QB
   int queries_per_wg;     // queries owned by one epilogue warpgroup
   int groups;             // epilogue warpgroups per CTA
@@ -73,6 +77,13 @@ cudaError_t launch_pool_keys(const void* k, int64_t n_pools, int D, const void* 
 cudaError_t launch_prune_setup(const void* q, const float* w, const float* q_scale, bool fp8, int64_t S, int H,
                                int D, const void* keys, int64_t n_keys, float* pq, float* knorm,
                                cudaStream_t stream);
+// Upper bound of key-range splits per query block (the merge keeps its
+// per-split offsets in shared memory).
+constexpr int kMaxSplits = 512;
+
+cudaError_t launch_merge_splits(int64_t S, int64_t q_pos0, int splits, int ksel, int width, int out_ratio,
+                                const uint2* split_buf, const int32_t* split_cnt, uint2* gather,
+                                int64_t gather_stride, int32_t* out_idx, int32_t* out_len, float* out_score, cudaStream_t stream);
 cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
                                 int32_t* shared, int32_t* left, int32_t* right, int32_t* counts,
                                 cudaStream_t stream);

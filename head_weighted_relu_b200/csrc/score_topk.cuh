@@ -151,6 +151,29 @@ __device__ __forceinline__ int tiles_of_block(const ScoreParams& p, int b) {
   return (n + kBM - 1) / kBM;
 }
 
+// A CTA's work item: query block b, key tiles [j0, j1) of it, split index sp.
+// With few query blocks (decode-like shapes) each block's key tiles are cut
+// into p.splits consecutive ranges, each its own item; the per-split top-K
+// lists are merged afterwards.  b < 0 once this CTA is done.
+struct Item {
+  int b, j0, j1, sp;
+};
+template <int QB, bool SPLIT>
+__device__ __forceinline__ Item item_of(const ScoreParams& p, int round, int cta, int grid) {
+  if constexpr (!SPLIT) {
+    const int b = block_of(round, cta, grid, p.n_blocks);
+    return {b, 0, b < 0 ? 0 : tiles_of_block<QB>(p, b), 0};
+  }
+  const int it = block_of(round, cta, grid, p.n_blocks * p.splits);
+  if (it < 0) return {-1, 0, 0, 0};
+  const int b = it / p.splits;
+  const int sp = it - b * p.splits;
+  const int nt = tiles_of_block<QB>(p, b);
+  const int per = (nt + p.splits - 1) / p.splits;
+  const int j0 = min(sp * per, nt);
+  return {b, j0, min(j0 + per, nt), sp};
+}
+
 // 2 * max(x, 0) for two accumulator columns, computed as x + |x| with one
 // packed add (exact: 2x for x >= 0, +0 otherwise).  The head weights are
 // staged halved (also exact), so w/2 * (x + |x|) rounds exactly like
@@ -585,7 +608,7 @@ __device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
-template <int H, int D, bool FP8, bool PRUNE>
+template <int H, int D, bool FP8, bool PRUNE, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const ScoreParams p) {
@@ -647,10 +670,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kph = 0, qe_ph = 0;
       bool first = true, ok = true;
       for (int r = 0; ok; ++r) {
-        const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
+        const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+        const int b = it.b;
         if (b < 0) break;
-        const int nt = tiles_of_block<QB>(p, b);
-        if (nt == 0) continue;
+        if (it.j1 == it.j0) continue;
         if (!first) {
           ok = mbar_wait(&bars->qempty, qe_ph, abort_flag, kWaitLimitNs);
           qe_ph ^= 1;
@@ -661,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_2d(smem + C::OFF_Q + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS, b * QB * H, &bars->qfull);
-        for (int j = 0; j < nt; ++j) {
+        for (int j = it.j0; j < it.j1; ++j) {
           ok = mbar_wait(&bars->kempty[stage], kph ^ 1u, abort_flag, kWaitLimitNs);
           if (!ok) break;
           mbar_arrive_expect_tx(&bars->kfull[stage], C::K_STAGE_BYTES);
@@ -691,9 +714,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t tcount = 0;  // tiles issued so far; tile n goes to accumulator n & 1
       bool ok = true;
       for (int r = 0; ok; ++r) {
-        const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
-        if (b < 0) break;
-        const int nt = tiles_of_block<QB>(p, b);
+        const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+        if (it.b < 0) break;
+        const int nt = it.j1 - it.j0;
         if (nt == 0) continue;
         ok = mbar_wait(&bars->qfull, qf_ph, abort_flag, kWaitLimitNs);
         qf_ph ^= 1u;
@@ -762,9 +785,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool failed = false;
     unsigned long long n_screened = 0ull, n_bounded = 0ull, n_skipped = 0ull;  // pruning counters (lane 0)
     for (int r = 0; !failed; ++r) {
-      const int b = block_of(r, blockIdx.x, gridDim.x, p.n_blocks);
+      const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+      const int b = it.b;
       if (b < 0) break;
-      const int nt = tiles_of_block<QB>(p, b);
+      const int nt = it.j1;
       const int64_t tq0 = static_cast<int64_t>(b) * QB + eg * NQW;
       uint2* cand = p.cand + (static_cast<size_t>(blockIdx.x) * kEpiGroups + eg) * NQW * static_cast<size_t>(p.cap);
 
@@ -798,7 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // to overflow or the block's tiles are done; the selection steps (cut of
       // the full buffers, or the final top-K of every query) follow it, so the
       // per-tile path carries none of their code.
-      int j = 0;
+      int j = it.j0;
       while (true) {
         // the group's head weights, in registers for the whole tile loop when
         // they fit (reloaded after a cut, which needs the registers)
@@ -814,8 +838,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         auto wget = [&](int col) -> float2 {
-          if (col < kWsm) return *reinterpret_cast<const float2*>(wsm + col);
-          return make_float2(wr[col - kWsm], wr[col - kWsm + 1]);
+          if constexpr (kWsm < C::CW) {
+            if (col >= kWsm) return make_float2(wr[col - kWsm], wr[col - kWsm + 1]);
+          }
+          return *reinterpret_cast<const float2*>(wsm + col);
         };
         // per-query state that only the selection steps change, in registers
         // for the tile loop: candidates held, threshold, visible keys
@@ -994,7 +1020,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             int32_t* orow = p.out_idx + t * p.width;
             float* srow = p.out_score ? p.out_score + t * p.width : nullptr;
             const int m = p.out_ratio;
+            // with split key ranges this is one split's top-K, kept as
+            // (ordered score, key) pairs in key order for the merge
+            uint2* srow_split = nullptr;
+            if constexpr (SPLIT) srow_split = p.split_buf + (static_cast<size_t>(t) * p.splits + it.sp) * p.ksel;
             auto emit = [&](int pos, uint32_t k, uint32_t ix) {
+              if constexpr (SPLIT) {
+                srow_split[pos] = make_uint2(k, ix);
+                return;
+              }
               const float sc = key_to_float(k);
               if (m == 1) {
                 orow[pos] = static_cast<int32_t>(ix);
@@ -1018,6 +1052,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
               kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id,
                                 [&](int pos, uint2 e) { emit(pos, e.x, e.y); });
+            }
+            if constexpr (SPLIT) {
+              if (etid == 0) p.split_cnt[t * p.splits + it.sp] = kept;
+              named_bar(bar_id, kBM);
+              continue;
             }
             int len = kept * m;
             if (m > 1) {
@@ -1061,7 +1100,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int H, int D, bool FP8, bool PRUNE>
 void fill_variant(ScoreVariant* v) {
   using C = Cfg<H, D, FP8>;
-  v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8, PRUNE>);
+  v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8, PRUNE, false>);
+  v->fn_split = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8, PRUNE, true>);
   v->queries_per_block = C::QB;
   v->queries_per_wg = C::NQW;
   v->groups = kEpiGroups;

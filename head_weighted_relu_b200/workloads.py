@@ -19,6 +19,10 @@ Workloads (names carry their sizes):
   long_1m_fp8       T=1,048,576 keys, the last 16,384 positions as queries,
                     H=64, D=128, K=2,048, FP8 e4m3 q and k with per-row FP32
                     scales (amax / 448).
+  decode_1m_s16     16 query rows at the end of T=1,048,576 keys (a decode step
+                    of 16 sequences' worth of indexer queries against one long
+                    context), H=64, D=128, K=2,048, bf16: the split key-range
+                    path.  Not one of the configurations the pages quote.
 """
 
 from __future__ import annotations
@@ -72,6 +76,8 @@ WORKLOADS = {
     "long_1m_fp8": Workload("long_1m_fp8", S=16384, T=1048576, H=64, D=128,
                             K=2048, dtype="fp8", q_pos0=1048576 - 16384,
                             seed=4, pair_overlap=True),
+    "decode_1m_s16": Workload("decode_1m_s16", S=16, T=1048576, H=64, D=128,
+                              K=2048, q_pos0=1048576 - 16, seed=6),
 }
 
 
