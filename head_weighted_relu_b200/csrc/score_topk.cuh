@@ -1041,20 +1041,26 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             };
             int kept;
+            [[maybe_unused]] uint32_t kth = 0u;  // ordered score of the K-th entry kept (0: fewer than K)
             if (n <= kRegCap) {
               RegBuf rb;
               rb_load(rb, buf, n, etid);
               RegCut c{0u, 0xFFFFFFFFu, false, n};
               if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
               kept = rb_compact(rb, n, c, all, st->scan, etid, bar_id, emit);
+              if constexpr (SPLIT) kth = all ? 0u : c.v;
             } else {
               Cut cut{0u, 0xFFFFFFFFu};
               if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
+              if constexpr (SPLIT) kth = all ? 0u : cut.v;
               kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id,
                                 [&](int pos, uint2 e) { emit(pos, e.x, e.y); });
             }
             if constexpr (SPLIT) {
-              if (etid == 0) p.split_cnt[t * p.splits + it.sp] = kept;
+              if (etid == 0) {
+                p.split_cnt[t * p.splits + it.sp] = kept;
+                p.split_kth[t * p.splits + it.sp] = kth;
+              }
               named_bar(bar_id, kBM);
               continue;
             }
