@@ -74,7 +74,7 @@ struct Plan {
   size_t split_bytes;      // per-split top-K lists
   int64_t gather_stride;   // entries per query of the merge's gathered list (a multiple of 128)
   size_t gather_bytes;
-  size_t split_cnt_bytes;  // per-split list lengths and K-th scores
+  size_t split_cnt_bytes;  // per-split list lengths, K-th and r-th scores
   size_t ws_bytes;
 };
 
@@ -142,7 +142,7 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
       // inside the query's own region
       pl->gather_stride = (static_cast<int64_t>(pl->splits) * pl->ksel + 127) / 128 * 128;
       pl->gather_bytes = align256(static_cast<size_t>(p->S) * pl->gather_stride * sizeof(uint2));
-      pl->split_cnt_bytes = 2 * align256(static_cast<size_t>(p->S) * pl->splits * sizeof(int32_t));
+      pl->split_cnt_bytes = 3 * align256(static_cast<size_t>(p->S) * pl->splits * sizeof(int32_t));
     }
   }
   pl->kp_bytes = p->visibility == INDEXER_VIS_POOLED
@@ -244,7 +244,9 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   uint2* split_gather = reinterpret_cast<uint2*>(split_base + pl.split_bytes);
   int32_t* split_cnt = reinterpret_cast<int32_t*>(split_base + pl.split_bytes + pl.gather_bytes);
   uint32_t* split_kth =
-      reinterpret_cast<uint32_t*>(split_base + pl.split_bytes + pl.gather_bytes + pl.split_cnt_bytes / 2);
+      reinterpret_cast<uint32_t*>(split_base + pl.split_bytes + pl.gather_bytes + pl.split_cnt_bytes / 3);
+  uint32_t* split_rth =
+      reinterpret_cast<uint32_t*>(split_base + pl.split_bytes + pl.gather_bytes + 2 * (pl.split_cnt_bytes / 3));
   // status word and the three pruning counters (bytes 0, 8, 16, 24) start at zero
   if (cudaMemsetAsync(status, 0, 32, stream) != cudaSuccess) return INDEXER_ECUDA;
   if (p->S == 0) return INDEXER_OK;
@@ -289,6 +291,7 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   sp.split_buf = split_buf;
   sp.split_cnt = split_cnt;
   sp.split_kth = split_kth;
+  sp.split_rth = split_rth;
   if (pl.prune && launch_prune_setup(q, w, q_scale, fp8, p->S, p->H, p->D, keys, pl.n_keys, pq, knorm,
                                      stream) != cudaSuccess)
     return INDEXER_ECUDA;
@@ -301,7 +304,7 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
     return INDEXER_ECUDA;
   if (pl.splits > 1 &&
       launch_merge_splits(p->S, p->q_pos0, pl.splits, pl.ksel, pl.width, pl.out_ratio, split_buf, split_cnt,
-                          split_kth, split_gather, pl.gather_stride, out_idx, out_len, out_score,
+                          split_kth, split_rth, split_gather, pl.gather_stride, out_idx, out_len, out_score,
                           stream) != cudaSuccess)
     return INDEXER_ECUDA;
   return INDEXER_OK;

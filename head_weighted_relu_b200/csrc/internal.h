@@ -43,6 +43,8 @@ struct ScoreParams {
   uint2* split_buf;      // splits > 1: [S][splits][ksel] top-K of each split, in key order
   int32_t* split_cnt;    // splits > 1: [S][splits] entries of each split
   uint32_t* split_kth;   // splits > 1: [S][splits] ordered score of each full split's K-th entry, else 0
+  uint32_t* split_rth;   // splits > 1: [S][splits] ordered score of each split's r-th entry, r = ceil(K / splits)
+                         // (0 when it has fewer than r)
 };
 
 // Per-variant launch facts, filled by the kernel's translation unit.
@@ -84,7 +86,7 @@ constexpr int kMaxSplits = 512;
 
 cudaError_t launch_merge_splits(int64_t S, int64_t q_pos0, int splits, int ksel, int width, int out_ratio,
                                 const uint2* split_buf, const int32_t* split_cnt, const uint32_t* split_kth,
-                                uint2* gather, int64_t gather_stride, int32_t* out_idx, int32_t* out_len,
+                                const uint32_t* split_rth, uint2* gather, int64_t gather_stride, int32_t* out_idx, int32_t* out_len,
                                 float* out_score, cudaStream_t stream);
 cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
                                 int32_t* shared, int32_t* left, int32_t* right, int32_t* counts,

@@ -1042,17 +1042,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             int kept;
             [[maybe_unused]] uint32_t kth = 0u;  // ordered score of the K-th entry kept (0: fewer than K)
+            [[maybe_unused]] uint32_t rth = 0u;  // split ranges: ordered score of the r-th entry (0: fewer)
             if (n <= kRegCap) {
               RegBuf rb;
               rb_load(rb, buf, n, etid);
               RegCut c{0u, 0xFFFFFFFFu, false, n};
               if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
               kept = rb_compact(rb, n, c, all, st->scan, etid, bar_id, emit);
-              if constexpr (SPLIT) kth = all ? 0u : c.v;
+              if constexpr (SPLIT) {
+                kth = all ? 0u : c.v;
+                // the r-th largest score of the range, r = ceil(K / splits)
+                const int r = (p.ksel + p.splits - 1) / p.splits;
+                if (n >= r)
+                  rth = rb_cut(rb, n, static_cast<uint32_t>(r), false, 0, hist, st->red, etid, bar_id).v;
+              }
             } else {
               Cut cut{0u, 0xFFFFFFFFu};
               if (!all) cut = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
-              if constexpr (SPLIT) kth = all ? 0u : cut.v;
+              if constexpr (SPLIT) {
+                kth = all ? 0u : cut.v;
+                const int r = (p.ksel + p.splits - 1) / p.splits;
+                if (n >= r)
+                  rth = wg_radix_select(buf, n, static_cast<uint32_t>(r), false, false, 0u,
+                                        static_cast<uint32_t>(n), hist, st->red, etid, bar_id).v;
+              }
               kept = wg_compact(buf, n, cut, all, &st->cwc[0][0], etid, bar_id,
                                 [&](int pos, uint2 e) { emit(pos, e.x, e.y); });
             }
@@ -1060,6 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (etid == 0) {
                 p.split_cnt[t * p.splits + it.sp] = kept;
                 p.split_kth[t * p.splits + it.sp] = kth;
+                p.split_rth[t * p.splits + it.sp] = rth;
               }
               named_bar(bar_id, kBM);
               continue;
