@@ -29,6 +29,8 @@ def _outputs(prob, device):
     W.Workload("tok", S=2000, T=2000, H=64, D=128, K=256, seed=41),
     W.Workload("pool", S=1500, T=1500, H=32, D=128, K=128, visibility=W.POOLED, ratio=4, seed=42),
     W.Workload("fp8", S=200, T=3000, H=64, D=128, K=300, dtype="fp8", q_pos0=2800, seed=43),
+    # few query rows against many keys: key ranges split across CTAs, then merged
+    W.Workload("decode", S=8, T=40000, H=64, D=128, K=512, q_pos0=40000 - 8, seed=44),
 ], ids=lambda w: w.name)
 def test_noalloc_matches_workspace_entry_point(cuda_ok, wl):
     from head_weighted_relu_b200 import indexer as I
