@@ -90,3 +90,18 @@ def test_decode_matches_unsplit_shape(cuda_ok):
     g_big = parity.run_gpu(big, inp, with_scores=False)
     g_small = parity.run_gpu(small, sub, with_scores=False)
     assert torch.equal(g_big[0][-4:], g_small[0]) and torch.equal(g_big[1][-4:], g_small[1])
+
+
+@pytest.mark.parametrize("wl", [
+    # a budget above the register-resident selection: the ranges and the merge
+    # select on global memory
+    W.Workload("dec_kbig", S=4, T=100000, H=64, D=128, K=4096, q_pos0=100000 - 4, seed=59),
+    # 32 query rows per block (4 heads) over a key count that ends mid-tile
+    W.Workload("dec_h4", S=40, T=33333, H=4, D=64, K=100, q_pos0=33333 - 40, seed=60),
+], ids=lambda w: w.name)
+def test_decode_edge_shapes(cuda_ok, wl):
+    assert _splits(wl) > 1
+    inp = W.generate(wl, "cuda")
+    gpu = parity.run_gpu(wl, inp)
+    recall = parity.assert_tolerant(wl, gpu, parity.oracle_rows(wl, inp, _rows(wl)), _rows(wl))
+    assert recall >= 0.9999
