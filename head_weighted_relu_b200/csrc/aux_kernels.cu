@@ -88,9 +88,51 @@ cudaError_t launch_pool_keys(const void* k, int64_t n_pools, int D, const void* 
 }
 
 // One warp per pair: each lane takes entries of A and binary-searches B.
+// Rows up to this width are searched in shared memory (one row per warp at a
+// time): a search step then costs a shared-memory access instead of an L2
+// round trip.  2,304 covers budgets of 2,048 and the pooled 2,051 slots.
+constexpr int kPairSmemRow = 2304;
+constexpr int kPairWarps = 4;
+
+// Copies row[0, n) to the warp's shared-memory slot and returns it, or returns
+// the row itself when it is wider than the slot.
+__device__ __forceinline__ const int32_t* stage_row(const int32_t* __restrict__ row, int n, int32_t* slot,
+                                                    int lane) {
+  if (n > kPairSmemRow) return row;
+#pragma unroll 4
+  for (int i = lane; i < n; i += 32) slot[i] = row[i];
+  __syncwarp();
+  return slot;
+}
+
+// Entries per lane and step in the pair kernels: four loads and four
+// searches in flight hide the load latency.
+constexpr int kPairILP = 4;
+
+// hit[u] = the strictly ascending row b[0, lb) holds x[u].  The four searches
+// advance together (binary lifting: pos counts the entries below x), so their
+// shared-memory reads overlap.
+__device__ __forceinline__ void rows_hold(const int32_t* __restrict__ b, int lb, const int32_t (&x)[kPairILP],
+                                          bool (&hit)[kPairILP]) {
+  int pos[kPairILP];
+#pragma unroll
+  for (int u = 0; u < kPairILP; ++u) pos[u] = 0;
+  for (int step = lb > 0 ? (1 << (31 - __clz(lb))) : 0; step > 0; step >>= 1) {
+#pragma unroll
+    for (int u = 0; u < kPairILP; ++u) {
+      const int c = pos[u] + step;
+      if (c <= lb && b[c - 1] < x[u]) pos[u] = c;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kPairILP; ++u) hit[u] = pos[u] < lb && b[pos[u]] == x[u];
+}
+
 __global__ void pair_overlap_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ len,
                                     int64_t n_pairs, int width, int32_t* __restrict__ out) {
+  __shared__ int32_t rows_s[kPairWarps][kPairSmemRow];
   const int lane = threadIdx.x & 31;
+  int32_t* slot = rows_s[threadIdx.x >> 5];
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t pr = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); pr < n_pairs;
        pr += warps) {
@@ -98,35 +140,24 @@ __global__ void pair_overlap_kernel(const int32_t* __restrict__ idx, const int32
     const int32_t* b = idx + (2 * pr + 1) * width;
     const int la = min(max(len[2 * pr], 0), width);
     const int lb = min(max(len[2 * pr + 1], 0), width);
+    const int32_t* bs = stage_row(b, lb, slot, lane);
     int count = 0;
-    for (int i = lane; i < la; i += 32) {
-      const int32_t x = a[i];
-      int lo = 0, hi = lb;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (b[mid] < x)
-          lo = mid + 1;
-        else
-          hi = mid;
+    for (int base = 0; base < la; base += 32 * kPairILP) {
+      int32_t x[kPairILP];
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) {
+        const int i = base + u * 32 + lane;
+        x[u] = i < la ? a[i] : 0;
       }
-      count += (lo < lb && b[lo] == x) ? 1 : 0;
+      bool hit[kPairILP];
+      rows_hold(bs, lb, x, hit);
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) count += (base + u * 32 + lane < la && hit[u]) ? 1 : 0;
     }
     count = warp_sum_i32(count);
     if (lane == 0) out[pr] = count;
+    __syncwarp();  // the slot is restaged for the next pair
   }
-}
-
-// True when the strictly ascending row b[0, lb) holds x (binary search).
-__device__ __forceinline__ bool row_holds(const int32_t* __restrict__ b, int lb, int32_t x) {
-  int lo = 0, hi = lb;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (b[mid] < x)
-      lo = mid + 1;
-    else
-      hi = mid;
-  }
-  return lo < lb && b[lo] == x;
 }
 
 // One warp per pair.  The rows are ascending, so taking a row's entries in
@@ -137,8 +168,10 @@ __global__ void pair_regions_kernel(const int32_t* __restrict__ idx, const int32
                                     int64_t n_pairs, int width, int32_t* __restrict__ shared,
                                     int32_t* __restrict__ left, int32_t* __restrict__ right,
                                     int32_t* __restrict__ counts) {
+  __shared__ int32_t rows_s[kPairWarps][kPairSmemRow];
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
+  int32_t* slot = rows_s[threadIdx.x >> 5];
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t pr = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5); pr < n_pairs;
        pr += warps) {
@@ -146,28 +179,52 @@ __global__ void pair_regions_kernel(const int32_t* __restrict__ idx, const int32
     const int32_t* b = idx + (2 * pr + 1) * width;
     const int la = min(max(len[2 * pr], 0), width);
     const int lb = min(max(len[2 * pr + 1], 0), width);
+    const int32_t* bs = stage_row(b, lb, slot, lane);
     int32_t* so = shared + pr * width;
     int32_t* lo = left + pr * width;
     int32_t* ro = right + pr * width;
     int ns = 0, nl = 0, nr = 0;
-    for (int base = 0; base < la; base += 32) {
-      const int i = base + lane;
-      const bool in = i < la;
-      const int32_t x = in ? a[i] : 0;
-      const bool both = in && row_holds(b, lb, x);
-      const uint32_t bs = __ballot_sync(kFullMask, both);
-      const uint32_t bl = __ballot_sync(kFullMask, in && !both);
-      if (both) so[ns + __popc(bs & lt)] = x;
-      if (in && !both) lo[nl + __popc(bl & lt)] = x;
-      ns += __popc(bs);
-      nl += __popc(bl);
+    for (int base = 0; base < la; base += 32 * kPairILP) {
+      int32_t x[kPairILP];
+      bool both[kPairILP];
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) {
+        const int i = base + u * 32 + lane;
+        x[u] = i < la ? a[i] : 0;
+      }
+      rows_hold(bs, lb, x, both);
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) both[u] = both[u] && base + u * 32 + lane < la;
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) {  // groups of 32 in row order keep each region ascending
+        const bool in = base + u * 32 + lane < la;
+        const uint32_t bsh = __ballot_sync(kFullMask, both[u]);
+        const uint32_t bl = __ballot_sync(kFullMask, in && !both[u]);
+        if (both[u]) so[ns + __popc(bsh & lt)] = x[u];
+        if (in && !both[u]) lo[nl + __popc(bl & lt)] = x[u];
+        ns += __popc(bsh);
+        nl += __popc(bl);
+      }
     }
-    for (int base = 0; base < lb; base += 32) {
-      const int i = base + lane;
-      const bool only = i < lb && !row_holds(a, la, b[i]);
-      const uint32_t br = __ballot_sync(kFullMask, only);
-      if (only) ro[nr + __popc(br & lt)] = b[i];
-      nr += __popc(br);
+    __syncwarp();  // every lane is done with the staged right row
+    const int32_t* as = stage_row(a, la, slot, lane);
+    for (int base = 0; base < lb; base += 32 * kPairILP) {
+      int32_t x[kPairILP];
+      bool only[kPairILP];
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) {
+        const int i = base + u * 32 + lane;
+        x[u] = i < lb ? b[i] : 0;
+      }
+      rows_hold(as, la, x, only);
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) only[u] = !only[u] && base + u * 32 + lane < lb;
+#pragma unroll
+      for (int u = 0; u < kPairILP; ++u) {
+        const uint32_t br = __ballot_sync(kFullMask, only[u]);
+        if (only[u]) ro[nr + __popc(br & lt)] = x[u];
+        nr += __popc(br);
+      }
     }
     for (int i = ns + lane; i < width; i += 32) so[i] = -1;
     for (int i = nl + lane; i < width; i += 32) lo[i] = -1;
@@ -177,6 +234,7 @@ __global__ void pair_regions_kernel(const int32_t* __restrict__ idx, const int32
       counts[3 * pr + 1] = nl;
       counts[3 * pr + 2] = nr;
     }
+    __syncwarp();  // the slot is restaged for the next pair
   }
 }
 
@@ -187,8 +245,8 @@ cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int threads = 256;  // 8 pairs per block
-  int64_t blocks = (n_pairs + 7) / 8;
+  const int threads = 32 * kPairWarps;  // one pair per warp at a time
+  int64_t blocks = (n_pairs + kPairWarps - 1) / kPairWarps;
   if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
   pair_regions_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, len, n_pairs, width, shared,
                                                                             left, right, counts);
@@ -201,8 +259,8 @@ cudaError_t launch_pair_overlap(const int32_t* idx, const int32_t* len, int64_t 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int threads = 256;  // 8 pairs per block
-  int64_t blocks = (n_pairs + 7) / 8;
+  const int threads = 32 * kPairWarps;  // one pair per warp at a time
+  int64_t blocks = (n_pairs + kPairWarps - 1) / kPairWarps;
   if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
   pair_overlap_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, len, n_pairs, width, out);
   return cudaGetLastError();
