@@ -211,10 +211,17 @@ indexer_status indexer_workspace_bytes(const indexer_problem* p, size_t* bytes) 
   return INDEXER_OK;
 }
 
-indexer_status indexer_topk(const indexer_problem* p, const void* q, const void* k, const float* w,
-                            const float* q_scale, const float* k_scale, const void* pool_coef, int32_t* out_idx,
-                            int32_t* out_len, float* out_score, void* workspace, size_t workspace_bytes,
-                            void* stream_) {
+}  // extern "C"
+
+namespace hwr {
+namespace {
+
+// indexer_topk; reset_status = false leaves the device status word as it is
+// (the host pipeline resets it once and runs one call per chunk of rows).
+indexer_status run_topk(const indexer_problem* p, const void* q, const void* k, const float* w,
+                        const float* q_scale, const float* k_scale, const void* pool_coef, int32_t* out_idx,
+                        int32_t* out_len, float* out_score, void* workspace, size_t workspace_bytes,
+                        void* stream_, bool reset_status) {
   Plan pl;
   indexer_status st = make_plan(p, true, &pl);
   if (st != INDEXER_OK) return st;
@@ -248,7 +255,7 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   uint32_t* split_rth =
       reinterpret_cast<uint32_t*>(split_base + pl.split_bytes + pl.gather_bytes + 2 * (pl.split_cnt_bytes / 3));
   // status word and the three pruning counters (bytes 0, 8, 16, 24) start at zero
-  if (cudaMemsetAsync(status, 0, 32, stream) != cudaSuccess) return INDEXER_ECUDA;
+  if (reset_status && cudaMemsetAsync(status, 0, 32, stream) != cudaSuccess) return INDEXER_ECUDA;
   if (p->S == 0) return INDEXER_OK;
 
   const void* keys = k;
@@ -310,6 +317,19 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
   return INDEXER_OK;
 }
 
+}  // namespace
+}  // namespace hwr
+
+extern "C" {
+
+indexer_status indexer_topk(const indexer_problem* p, const void* q, const void* k, const float* w,
+                            const float* q_scale, const float* k_scale, const void* pool_coef, int32_t* out_idx,
+                            int32_t* out_len, float* out_score, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  return hwr::run_topk(p, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len, out_score, workspace,
+                       workspace_bytes, stream, true);
+}
+
 indexer_status indexer_pool_keys(const void* k, int64_t T_tokens, int32_t D, const void* pool_coef,
                                  int32_t ratio, void* out_kp, void* stream) {
   if (!k || !pool_coef || !out_kp || T_tokens < 0 || D < 1 || D > 4096 || ratio < 1 || ratio > 16)
@@ -362,6 +382,196 @@ indexer_status indexer_read_status(void* workspace, int32_t* flags, void* stream
   if (cudaStreamSynchronize(s) != cudaSuccess) return INDEXER_ECUDA;
   *flags = static_cast<int32_t>(v);
   return INDEXER_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------
+// indexer_topk on host buffers: keys copied once, query rows streamed through
+// the device in chunks so that the copies overlap the indexer.
+// ------------------------------------------------------------------------
+namespace hwr {
+namespace {
+
+struct HostLayout {
+  int64_t chunk;         // query rows per chunk
+  int64_t n_chunks;
+  size_t elem;           // bytes per q / k element
+  size_t q_row, w_row;   // bytes of one query row of q, and of w (and of q_scale)
+  int32_t width;
+  size_t topk_ws;        // indexer workspace for one chunk (first, so its status word is at offset 0)
+  size_t off_k, off_ks, off_pc, off_slot;
+  size_t slot;           // bytes of one chunk slot: q, w, q_scale, idx, len, score rows
+  size_t s_w, s_qs, s_idx, s_len, s_sc;  // offsets inside a slot
+  size_t total;
+};
+
+indexer_problem chunk_problem(const indexer_problem* p, int64_t first, int64_t rows) {
+  indexer_problem c = *p;
+  c.S = rows;
+  c.q_pos0 = p->q_pos0 + first;
+  return c;
+}
+
+indexer_status host_layout(const indexer_problem* p, HostLayout* L) {
+  if (!p || p->S < 0) return INDEXER_EINVAL;
+  // about eight chunks, each large enough to fill the GPU on its own
+  const int64_t target = (p->S + 7) / 8;
+  int64_t chunk = target < 4096 ? 4096 : (target + 127) / 128 * 128;
+  if (chunk > p->S) chunk = p->S > 0 ? p->S : 1;
+  L->chunk = chunk;
+  L->n_chunks = p->S > 0 ? (p->S + chunk - 1) / chunk : 0;
+  L->elem = p->dtype == INDEXER_FP8_E4M3 ? 1 : 2;
+  L->q_row = static_cast<size_t>(p->H) * p->D * L->elem;
+  L->w_row = static_cast<size_t>(p->H) * sizeof(float);
+  int32_t width = 0;
+  indexer_status st = indexer_out_width(p, &width);
+  if (st != INDEXER_OK) return st;
+  L->width = width;
+  // every full chunk has the same shape; a shorter last chunk can plan
+  // differently (split key ranges), so both are sized
+  size_t ws = 0;
+  const int64_t last = L->n_chunks > 0 ? (L->n_chunks - 1) * chunk : 0;
+  for (int64_t first : {int64_t(0), last}) {
+    const int64_t rows = p->S - first < chunk ? p->S - first : chunk;
+    const indexer_problem c = chunk_problem(p, first, rows > 0 ? rows : 0);
+    size_t b = 0;
+    st = indexer_workspace_bytes(&c, &b);
+    if (st != INDEXER_OK) return st;
+    ws = b > ws ? b : ws;
+  }
+  L->topk_ws = align256(ws);
+  const bool fp8 = p->dtype == INDEXER_FP8_E4M3;
+  const bool pooled = p->visibility == INDEXER_VIS_POOLED;
+  L->off_k = L->topk_ws;
+  L->off_ks = L->off_k + align256(static_cast<size_t>(p->T) * p->D * L->elem);
+  L->off_pc = L->off_ks + (fp8 ? align256(static_cast<size_t>(p->T) * sizeof(float)) : 0);
+  L->off_slot = L->off_pc + (pooled ? align256(static_cast<size_t>(p->ratio) * p->D * 2) : 0);
+  const size_t c = static_cast<size_t>(chunk);
+  L->s_w = align256(c * L->q_row);
+  L->s_qs = L->s_w + align256(c * L->w_row);
+  L->s_idx = L->s_qs + (fp8 ? align256(c * L->w_row) : 0);
+  L->s_len = L->s_idx + align256(c * width * sizeof(int32_t));
+  L->s_sc = L->s_len + align256(c * sizeof(int32_t));
+  L->slot = L->s_sc + align256(c * width * sizeof(float));
+  L->total = L->off_slot + 2 * L->slot;
+  return INDEXER_OK;
+}
+
+}  // namespace
+}  // namespace hwr
+
+extern "C" {
+
+indexer_status indexer_host_workspace_bytes(const indexer_problem* p, size_t* bytes) {
+  HostLayout L;
+  const indexer_status st = host_layout(p, &L);
+  if (st != INDEXER_OK) return st;
+  if (!bytes) return INDEXER_EINVAL;
+  *bytes = L.total;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_topk_host(const indexer_problem* p, const void* q, const void* k, const float* w,
+                                 const float* q_scale, const float* k_scale, const void* pool_coef,
+                                 int32_t* out_idx, int32_t* out_len, float* out_score, void* workspace,
+                                 size_t workspace_bytes, void* stream_) {
+  HostLayout L;
+  indexer_status st = host_layout(p, &L);
+  if (st != INDEXER_OK) return st;
+  const bool fp8 = p->dtype == INDEXER_FP8_E4M3;
+  const bool pooled = p->visibility == INDEXER_VIS_POOLED;
+  if (!k || (p->S > 0 && (!q || !w || !out_idx || !out_len))) return INDEXER_EINVAL;
+  if (fp8 && (!q_scale || !k_scale)) return INDEXER_EINVAL;
+  if (pooled && !pool_coef) return INDEXER_EINVAL;
+  if (!workspace || !aligned(workspace, 256)) return INDEXER_EWORKSPACE;
+  if (workspace_bytes < L.total) return INDEXER_EWORKSPACE;
+  cudaStream_t sc = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // the status word and counters start at zero once for all chunks
+  if (cudaMemsetAsync(ws, 0, 32, sc) != cudaSuccess) return INDEXER_ECUDA;
+  if (p->S == 0) return INDEXER_OK;
+
+  // copies run on two streams of their own; events order them with the
+  // compute stream: a slot is refilled only after the indexer call that read
+  // it, and its results are overwritten only after they have been copied out
+  cudaStream_t sh = nullptr, sd = nullptr;
+  cudaEvent_t ev[8] = {};
+  auto cleanup = [&]() {
+    for (cudaEvent_t& e : ev)
+      if (e) cudaEventDestroy(e);
+    if (sh) cudaStreamDestroy(sh);
+    if (sd) cudaStreamDestroy(sd);
+  };
+  if (cudaStreamCreateWithFlags(&sh, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&sd, cudaStreamNonBlocking) != cudaSuccess) {
+    cleanup();
+    return INDEXER_ECUDA;
+  }
+  for (cudaEvent_t& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      cleanup();
+      return INDEXER_ECUDA;
+    }
+  cudaEvent_t ev_start = ev[0], ev_keys = ev[1];
+  cudaEvent_t ev_in[2] = {ev[2], ev[3]}, ev_done[2] = {ev[4], ev[5]}, ev_out[2] = {ev[6], ev[7]};
+  bool ok = true;
+  auto chk = [&](cudaError_t e) { ok = ok && e == cudaSuccess; };
+  // earlier work on the compute stream may still use the workspace
+  chk(cudaEventRecord(ev_start, sc));
+  chk(cudaStreamWaitEvent(sh, ev_start, 0));
+  chk(cudaStreamWaitEvent(sd, ev_start, 0));
+  chk(cudaMemcpyAsync(ws + L.off_k, k, static_cast<size_t>(p->T) * p->D * L.elem, cudaMemcpyHostToDevice, sh));
+  if (fp8)
+    chk(cudaMemcpyAsync(ws + L.off_ks, k_scale, static_cast<size_t>(p->T) * sizeof(float), cudaMemcpyHostToDevice,
+                        sh));
+  if (pooled)
+    chk(cudaMemcpyAsync(ws + L.off_pc, pool_coef, static_cast<size_t>(p->ratio) * p->D * 2, cudaMemcpyHostToDevice,
+                        sh));
+  chk(cudaEventRecord(ev_keys, sh));
+  chk(cudaStreamWaitEvent(sc, ev_keys, 0));
+  for (int64_t c = 0; ok && c < L.n_chunks; ++c) {
+    const int si = static_cast<int>(c & 1);
+    uint8_t* slot = ws + L.off_slot + si * L.slot;
+    const int64_t first = c * L.chunk;
+    const int64_t rows = p->S - first < L.chunk ? p->S - first : L.chunk;
+    // inputs of chunk c into slot si, once the call of chunk c - 2 is done with it
+    if (c >= 2) chk(cudaStreamWaitEvent(sh, ev_done[si], 0));
+    chk(cudaMemcpyAsync(slot, static_cast<const uint8_t*>(q) + first * L.q_row, rows * L.q_row,
+                        cudaMemcpyHostToDevice, sh));
+    chk(cudaMemcpyAsync(slot + L.s_w, w + first * p->H, rows * L.w_row, cudaMemcpyHostToDevice, sh));
+    if (fp8)
+      chk(cudaMemcpyAsync(slot + L.s_qs, q_scale + first * p->H, rows * L.w_row, cudaMemcpyHostToDevice, sh));
+    chk(cudaEventRecord(ev_in[si], sh));
+    // the indexer on chunk c, once its inputs are in and the results of
+    // chunk c - 2 have left slot si
+    chk(cudaStreamWaitEvent(sc, ev_in[si], 0));
+    if (c >= 2) chk(cudaStreamWaitEvent(sc, ev_out[si], 0));
+    if (!ok) break;
+    const indexer_problem cp = chunk_problem(p, first, rows);
+    st = run_topk(&cp, slot, ws + L.off_k, reinterpret_cast<const float*>(slot + L.s_w),
+                  fp8 ? reinterpret_cast<const float*>(slot + L.s_qs) : nullptr,
+                  fp8 ? reinterpret_cast<const float*>(ws + L.off_ks) : nullptr, pooled ? ws + L.off_pc : nullptr,
+                  reinterpret_cast<int32_t*>(slot + L.s_idx), reinterpret_cast<int32_t*>(slot + L.s_len),
+                  out_score ? reinterpret_cast<float*>(slot + L.s_sc) : nullptr, ws, L.topk_ws, sc, false);
+    if (st != INDEXER_OK) break;
+    chk(cudaEventRecord(ev_done[si], sc));
+    // results of chunk c to the host
+    chk(cudaStreamWaitEvent(sd, ev_done[si], 0));
+    chk(cudaMemcpyAsync(out_idx + first * L.width, slot + L.s_idx, rows * L.width * sizeof(int32_t),
+                        cudaMemcpyDeviceToHost, sd));
+    chk(cudaMemcpyAsync(out_len + first, slot + L.s_len, rows * sizeof(int32_t), cudaMemcpyDeviceToHost, sd));
+    if (out_score)
+      chk(cudaMemcpyAsync(out_score + first * L.width, slot + L.s_sc, rows * L.width * sizeof(float),
+                          cudaMemcpyDeviceToHost, sd));
+    chk(cudaEventRecord(ev_out[si], sd));
+  }
+  // the compute stream ends after the last copies out (the caller synchronises it)
+  chk(cudaEventRecord(ev_out[0], sd));
+  chk(cudaStreamWaitEvent(sc, ev_out[0], 0));
+  cleanup();
+  if (st != INDEXER_OK) return st;
+  return ok ? INDEXER_OK : INDEXER_ECUDA;
 }
 
 }  // extern "C"

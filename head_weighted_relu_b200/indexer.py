@@ -29,6 +29,7 @@ STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
 
 # every symbol include/hwr_indexer.h declares
 EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_topk_noalloc",
+           "indexer_host_workspace_bytes", "indexer_topk_host",
            "indexer_pool_keys",
            "indexer_pair_overlap", "indexer_pair_regions", "indexer_read_status", "indexer_read_prune_counters",
            "indexer_status_string",
@@ -62,6 +63,8 @@ def _load():
     lib.indexer_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
     lib.indexer_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.indexer_host_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+    lib.indexer_topk_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_pool_keys.argtypes = [vp, i64, i32, vp, i32, vp, vp]
     lib.indexer_pair_overlap.argtypes = [vp, vp, i64, i32, vp, vp]
     lib.indexer_pair_regions.argtypes = [vp, vp, i64, i32, vp, vp, vp, vp, vp]
@@ -121,6 +124,25 @@ def indexer_topk(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len
         ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
         _ptr(pool_coef), _ptr(out_idx), _ptr(out_len), _ptr(out_score), _ptr(workspace),
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def indexer_host_workspace_bytes(problem: Problem) -> int:
+    n = ctypes.c_size_t()
+    _check("indexer_host_workspace_bytes",
+           _lib.indexer_host_workspace_bytes(ctypes.byref(problem), ctypes.byref(n)))
+    return n.value
+
+
+def indexer_topk_host(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len, out_score,
+                      workspace, stream=None):
+    """indexer_topk on host tensors (pinned for the copies to overlap): inputs and
+    outputs live in host memory, `workspace` is a device buffer of
+    indexer_host_workspace_bytes bytes.  Ordered on `stream`; synchronise it
+    before reading the outputs."""
+    _check("indexer_topk_host", _lib.indexer_topk_host(
+        ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
+        _ptr(pool_coef), _ptr(out_idx), _ptr(out_len), _ptr(out_score), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def indexer_topk_noalloc(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len,

@@ -162,6 +162,30 @@ indexer_status indexer_topk_noalloc(const indexer_problem* p,
                                     int32_t* out_idx, int32_t* out_len, float* out_score,
                                     void* stream);
 
+/* indexer_topk on HOST buffers (page-locked for the copies to overlap):
+ * q, k, w, q_scale, k_scale and pool_coef are host pointers with the layouts
+ * of indexer_topk, and so are out_idx, out_len and out_score (NULL for none).
+ * The keys (with their scales or pool coefficients) are copied to the
+ * device once; the query rows then pass through it in chunks of a few
+ * thousand rows, the copy of chunk c+1's rows and of chunk c-1's results
+ * overlapping the indexer on chunk c.  Results equal indexer_topk's.
+ *   `workspace` is device memory of indexer_host_workspace_bytes bytes
+ *   (256-byte aligned): the indexer's workspace for one chunk first -- so
+ *   indexer_read_status applies to it, over all chunks -- then the keys and
+ *   two chunks of rows.
+ *   Asynchronous with respect to the host: the work is ordered on `stream`
+ *   (the copies run on two internal streams joined to it by events), and the
+ *   host buffers must stay valid until `stream` has been synchronised.  No
+ *   device memory is allocated; two streams and eight events are created and
+ *   released per call.  Errors as indexer_topk, plus INDEXER_ECUDA when a
+ *   copy or stream operation fails. */
+indexer_status indexer_host_workspace_bytes(const indexer_problem* p, size_t* bytes);
+indexer_status indexer_topk_host(const indexer_problem* p, const void* q, const void* k,
+                                 const float* w, const float* q_scale,
+                                 const float* k_scale, const void* pool_coef,
+                                 int32_t* out_idx, int32_t* out_len, float* out_score,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Pool formation alone (the first step of POOLED):
  *   kp[p, d] = RNE_bf16( exact sum_{j<ratio} c[j, d] * k[ratio*p + j, d] )
  * for p < T_tokens / ratio; k [T_tokens, D] bf16, pool_coef [ratio, D] bf16,
