@@ -415,8 +415,9 @@ indexer_problem chunk_problem(const indexer_problem* p, int64_t first, int64_t r
 
 indexer_status host_layout(const indexer_problem* p, HostLayout* L) {
   if (!p || p->S < 0) return INDEXER_EINVAL;
-  // about eight chunks, each large enough to fill the GPU on its own
-  const int64_t target = (p->S + 7) / 8;
+  // about sixteen chunks (a short first copy before the pipeline fills), each
+  // large enough to fill the GPU on its own
+  const int64_t target = (p->S + 15) / 16;
   int64_t chunk = target < 4096 ? 4096 : (target + 127) / 128 * 128;
   if (chunk > p->S) chunk = p->S > 0 ? p->S : 1;
   L->chunk = chunk;
