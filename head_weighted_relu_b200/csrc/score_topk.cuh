@@ -103,7 +103,7 @@ struct Cfg {
   // and two-query groups with 16 in registers (register pressure elsewhere).
   static constexpr bool WREG = NQW <= 2;
   static constexpr int WSM_COLS = !WREG ? CW : ((!FP8 && NQW == 1) ? 0 : 48);
-  static constexpr int CHAINS = 2;                       // packed partial sums per query (fewest registers)
+  static constexpr int CHAINS = FP8 ? 1 : 2;             // packed partial sums per query (FP8: fewest registers)
   static constexpr int Q_ACC_BYTES = BN * ROW_BYTES;
   static constexpr int Q_BYTES = Q_ACC_BYTES;
   static constexpr int K_STAGE_BYTES = kBM * ROW_BYTES;
@@ -206,8 +206,10 @@ template <int CHAINS>
 __device__ __forceinline__ float chain_total(const float2 (&a)[CHAINS]) {
   if constexpr (CHAINS == 4)
     return ((a[0].x + a[0].y) + (a[1].x + a[1].y)) + ((a[2].x + a[2].y) + (a[3].x + a[3].y));
-  else
+  else if constexpr (CHAINS == 2)
     return (a[0].x + a[0].y) + (a[1].x + a[1].y);
+  else
+    return a[0].x + a[0].y;
 }
 
 // Upper bound of a key's score from the first kPruneR heads of a query
