@@ -25,6 +25,7 @@ from .indexer_oracle import (  # noqa: F401
     select_topk,
     out_width,
     topk_rows,
+    topk_rows_docs,
     decode_keys_for,
     pair_shared_counts,
     pair_regions,

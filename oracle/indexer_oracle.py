@@ -317,6 +317,84 @@ def topk_rows(problem: dict, q_rows, k, w_rows, rows, q_scale_rows=None,
     return out_idx, out_len, out_score, taus
 
 
+def topk_rows_docs(problem: dict, q_rows, k, w_rows, rows, doc_bounds, q_scale_rows=None,
+                   k_scale=None, pool_coef=None):
+    """Indexer output for query rows of a packed batch of documents.
+
+    Token positions [doc_bounds[d], doc_bounds[d+1]) form document d; a query
+    sees only its own document, and pools never cross a document boundary
+    ("Module 06 — DSA & KPool: Selective Retrieval", §3 and "Ship it": in a
+    packed-document batch no pool may span a document boundary, and no token
+    of one document may reach another document's selection).  For the query at global
+    position g in document d starting at token b:
+      TOKEN       keys b .. g;
+      COMPRESSED  compressed keys j with j >= b / ratio and ratio*j+ratio-1 <= g
+                  (documents start on a multiple of the ratio);
+      POOLED      the document's pools: pool p covers tokens b+ratio*p ..
+                  b+ratio*p+ratio-1, its key pooled from those tokens, visible
+                  once complete; selected pools expand to their tokens, then
+                  the tokens b+ratio*nc .. g of the document's incomplete pool.
+    Indices are global token (or compressed-key) positions.  Arguments and
+    results as topk_rows.
+    """
+    vis_mode = problem["visibility"]
+    ratio = int(problem["ratio"]) if vis_mode != TOKEN else 1
+    K = int(problem["K"])
+    width = out_width(K, vis_mode, ratio)
+    ksel = K // ratio if vis_mode == POOLED else K
+    bounds = np.asarray(doc_bounds, dtype=np.int64)
+    R = len(rows)
+    out_idx = np.full((R, width), -1, dtype=np.int32)
+    out_len = np.zeros(R, dtype=np.int32)
+    out_score = np.full((R, width), math.nan, dtype=np.float64)
+    taus = np.full(R, math.nan, dtype=np.float64)
+    if vis_mode == POOLED:
+        tokens = None
+    else:
+        tokens = _decode_keys(problem, k, k_scale, pool_coef)
+    pooled_cache = {}
+    for r in range(R):
+        g = int(problem["q_pos0"]) + int(rows[r])
+        d = int(np.searchsorted(bounds, g, side="right")) - 1
+        b = int(bounds[d])
+        if problem["dtype"] == "fp8":
+            q_t = decode_e4m3(q_rows[r]) * np.asarray(q_scale_rows[r], dtype=np.float64)[:, None]
+        else:
+            q_t = decode_bf16(q_rows[r])
+        w_t = np.asarray(w_rows[r], dtype=np.float64)
+        if vis_mode == TOKEN:
+            vis = np.arange(b, g + 1, dtype=np.int64)
+            block = tokens[vis]
+        elif vis_mode == COMPRESSED:
+            j = np.arange(tokens.shape[0], dtype=np.int64)
+            vis = j[(j >= b // ratio) & (ratio * j + ratio - 1 <= g)]
+            block = tokens[vis]
+        else:
+            end = int(bounds[d + 1])
+            if d not in pooled_cache:
+                pooled_cache[d] = decode_bf16(pooled_keys(np.asarray(k)[b:end], pool_coef, ratio))
+            doc_pools = pooled_cache[d]
+            n_done = (g - b + 1) // ratio            # complete pools of the document
+            vis = np.arange(n_done, dtype=np.int64)  # document-local pool numbers
+            block = doc_pools[:n_done]
+        s = score_keys(q_t, w_t, block)
+        sel, ssel, tau = select_topk(s, vis, ksel)
+        taus[r] = tau
+        if vis_mode == POOLED:
+            pos = (b + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)
+            sc = np.repeat(ssel, ratio)
+            doc_tail = np.arange(b + ratio * n_done, g + 1, dtype=np.int64)
+            pos = np.concatenate((pos, doc_tail))
+            sc = np.concatenate((sc, np.full(doc_tail.size, math.nan)))
+        else:
+            pos, sc = sel, ssel
+        n = pos.size
+        out_idx[r, :n] = pos
+        out_len[r] = n
+        out_score[r, :n] = sc
+    return out_idx, out_len, out_score, taus
+
+
 def decode_keys_for(problem: dict, k, k_scale=None, pool_coef=None) -> np.ndarray:
     """Decoded float64 keys (pooled keys for POOLED) for reuse across calls."""
     return _decode_keys(problem, k, k_scale, pool_coef)

@@ -426,6 +426,54 @@ def pin_pair_regions(O):
     assert c[1, 1] == 0 and c[1, 2] == 0   # identical rows: nothing unique
 
 
+def pin_documents(O):
+    """Packed documents ("Module 06 — DSA & KPool", §3 and "Ship it"): one
+    document covering everything is the plain indexer; for token keys the
+    output equals a brute-force top-K of the full score row with every key
+    outside [document start, g] excluded; pooled output never leaves the
+    query's document, comes in whole pools aligned to the document start, and
+    ends with the document-relative incomplete tail."""
+    rng = np.random.default_rng(37)
+    H, D, T = 3, 8, 40
+    qb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, H, D)))
+    kb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, D)))
+    w = rng.integers(-2, 3, size=(T, H)).astype(np.float32)
+    rows = np.arange(T)
+    for vis, ratio, K in ((O.TOKEN, 1, 5), (O.POOLED, 4, 8)):
+        prob = _problem(S=T, T=T, H=H, D=D, K=K, vis=vis, ratio=ratio)
+        c = _bf16_bits_of_ints(rng.integers(0, 3, size=(ratio, D))) if vis == O.POOLED else None
+        a = O.topk_rows(prob, qb, kb, w, rows, pool_coef=c)
+        b = O.topk_rows_docs(prob, qb, kb, w, rows, [0, T], pool_coef=c)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    bounds = [0, 13, 14, 27, 40]   # a one-token document; lengths not multiples of 4
+    prob = _problem(S=T, T=T, H=H, D=D, K=5)
+    idx, ln, _, _ = O.topk_rows_docs(prob, qb, kb, w, rows, bounds)
+    keys = O.decode_bf16(kb)
+    for t in rows:
+        d = int(np.searchsorted(bounds, t, side="right")) - 1
+        s = O.score_keys(O.decode_bf16(qb[t]), w[t].astype(np.float64), keys)
+        s[: bounds[d]] = -np.inf
+        s[t + 1:] = -np.inf
+        n = min(5, t - bounds[d] + 1)
+        top = np.argsort(-s, kind="stable")[:n]
+        assert idx[t, : ln[t]].tolist() == sorted(top.tolist()), t
+    prob = _problem(S=T, T=T, H=H, D=D, K=8, vis=O.POOLED, ratio=4)
+    c = _bf16_bits_of_ints(rng.integers(0, 3, size=(4, D)))
+    idx, ln, _, _ = O.topk_rows_docs(prob, qb, kb, w, rows, bounds, pool_coef=c)
+    for t in rows:
+        d = int(np.searchsorted(bounds, t, side="right")) - 1
+        b = bounds[d]
+        row = idx[t, : ln[t]]
+        assert ((row >= b) & (row <= t)).all(), t
+        nc = (t - b + 1) // 4
+        tail = list(range(b + 4 * nc, t + 1))
+        body = row[: len(row) - len(tail)]
+        assert row[len(body):].tolist() == tail, t
+        assert len(body) % 4 == 0 and all((body[i] - b) % 4 == 0 and
+                                          body[i:i + 4].tolist() == list(range(body[i], body[i] + 4))
+                                          for i in range(0, len(body), 4)), t
+
+
 def pin_fp8_scales(O):
     """An FP8 value means code * row scale: doubling every key scale doubles
     every score and leaves the selection unchanged; a per-(query, head) scale
@@ -472,5 +520,6 @@ PINS = [
     pin_bf16_codec,
     pin_pair_overlap,
     pin_pair_regions,
+    pin_documents,
     pin_fp8_scales,
 ]

@@ -33,6 +33,10 @@ MUTATIONS = {
     "tail_before_pools": ("pos = np.concatenate([pos, tail])", "pos = np.concatenate([tail, pos])"),
     "regions_left_right_swapped": ("for r, members in enumerate((a & b, a - b, b - a)):",
                                    "for r, members in enumerate((a & b, b - a, a - b)):"),
+    "document_start_leaks": ("            vis = np.arange(b, g + 1, dtype=np.int64)",
+                             "            vis = np.arange(max(b - 1, 0), g + 1, dtype=np.int64)"),
+    "pools_from_global_grid": ("            pos = (b + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)",
+                               "            pos = (b // ratio * ratio + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)"),
     "regions_unsorted": ("            ordered = sorted(members)", "            ordered = sorted(members, reverse=True)"),
 }
 
