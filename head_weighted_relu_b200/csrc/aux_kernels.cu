@@ -253,6 +253,28 @@ cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t 
   return cudaGetLastError();
 }
 
+// Adds `add` to every valid index (>= 0) of n consecutive output entries: a
+// document's rows are computed with document-relative key numbers and then
+// shifted to global positions.
+__global__ void offset_indices_kernel(int32_t* __restrict__ idx, int64_t n, int32_t add) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int32_t v = idx[i];
+    if (v >= 0) idx[i] = v + add;
+  }
+}
+
+cudaError_t launch_offset_indices(int32_t* idx, int64_t n, int32_t add, cudaStream_t stream) {
+  if (n == 0 || add == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  offset_indices_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(idx, n, add);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_pair_overlap(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
                                 int32_t* out, cudaStream_t stream) {
   if (n_pairs == 0) return cudaSuccess;

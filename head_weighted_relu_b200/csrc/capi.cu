@@ -576,3 +576,130 @@ indexer_status indexer_topk_host(const indexer_problem* p, const void* q, const 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Packed-document batches: each document is its own indexer problem.
+// ------------------------------------------------------------------------
+namespace hwr {
+namespace {
+
+// Document d of a packed batch as an indexer problem on its own: its query
+// rows [r0, r0 + sub.S), its keys from key number key0, positions relative to
+// its first token.  `shift` turns its output indices into global ones.
+struct DocPart {
+  indexer_problem sub;
+  int64_t r0;
+  int64_t key0;
+  int32_t shift;
+};
+
+indexer_status doc_part(const indexer_problem* p, const int64_t* b, int32_t d, DocPart* out, bool* empty) {
+  const bool compressed = p->visibility == INDEXER_VIS_COMPRESSED;
+  const int64_t ratio = p->visibility == INDEXER_VIS_TOKEN ? 1 : p->ratio;
+  const int64_t lo = b[d], hi = b[d + 1];
+  int64_t r0 = lo - p->q_pos0, r1 = hi - p->q_pos0;
+  if (r0 < 0) r0 = 0;
+  if (r1 > p->S) r1 = p->S;
+  *empty = r1 <= r0;
+  out->sub = *p;
+  out->sub.S = *empty ? 0 : r1 - r0;
+  out->sub.q_pos0 = p->q_pos0 + r0 - lo;
+  out->sub.T = compressed ? (hi - lo) / ratio : hi - lo;
+  out->r0 = r0;
+  out->key0 = compressed ? lo / ratio : lo;
+  // token keys and pooled positions shift by the document's first token;
+  // compressed keys by its first compressed key
+  const int64_t shift = compressed ? lo / ratio : lo;
+  if (shift > INT32_MAX) return INDEXER_EUNSUPPORTED;
+  out->shift = static_cast<int32_t>(shift);
+  return INDEXER_OK;
+}
+
+// Bounds must rise strictly, cover every query position, stay within the
+// keys, and (compressed keys) start documents on a whole compressed key.
+indexer_status check_docs(const indexer_problem* p, const int64_t* b, int32_t n_docs) {
+  if (!p || !b || n_docs < 1) return INDEXER_EINVAL;
+  const bool compressed = p->visibility == INDEXER_VIS_COMPRESSED;
+  const int64_t ratio = p->visibility == INDEXER_VIS_TOKEN ? 1 : p->ratio;
+  if (ratio < 1) return INDEXER_EINVAL;
+  if (b[0] < 0) return INDEXER_EINVAL;
+  for (int32_t d = 0; d < n_docs; ++d) {
+    if (b[d + 1] <= b[d]) return INDEXER_EINVAL;
+    if (compressed && (b[d] % ratio != 0 || b[d + 1] % ratio != 0)) return INDEXER_EINVAL;
+  }
+  const int64_t key_tokens = compressed ? p->T * ratio : p->T;
+  if (b[n_docs] > key_tokens) return INDEXER_EINVAL;
+  if (p->S > 0 && (p->q_pos0 < b[0] || p->q_pos0 + p->S > b[n_docs])) return INDEXER_EINVAL;
+  return INDEXER_OK;
+}
+
+}  // namespace
+}  // namespace hwr
+
+extern "C" {
+
+indexer_status indexer_docs_workspace_bytes(const indexer_problem* p, const int64_t* doc_bounds, int32_t n_docs,
+                                            size_t* bytes) {
+  indexer_status st = check_docs(p, doc_bounds, n_docs);
+  if (st != INDEXER_OK) return st;
+  if (!bytes) return INDEXER_EINVAL;
+  size_t most = 0;
+  for (int32_t d = 0; d < n_docs; ++d) {
+    DocPart part;
+    bool empty = false;
+    st = doc_part(p, doc_bounds, d, &part, &empty);
+    if (st != INDEXER_OK) return st;
+    if (empty) continue;
+    size_t b = 0;
+    st = indexer_workspace_bytes(&part.sub, &b);
+    if (st != INDEXER_OK) return st;
+    most = b > most ? b : most;
+  }
+  *bytes = most > 256 ? most : 256;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_topk_docs(const indexer_problem* p, const void* q, const void* k, const float* w,
+                                 const float* q_scale, const float* k_scale, const void* pool_coef,
+                                 const int64_t* doc_bounds, int32_t n_docs, int32_t* out_idx, int32_t* out_len,
+                                 float* out_score, void* workspace, size_t workspace_bytes, void* stream) {
+  indexer_status st = check_docs(p, doc_bounds, n_docs);
+  if (st != INDEXER_OK) return st;
+  // pointers are checked here: per document they are offset before use
+  if (!k || (p->S > 0 && (!q || !w || !out_idx || !out_len))) return INDEXER_EINVAL;
+  if (p->dtype == INDEXER_FP8_E4M3 && (!q_scale || !k_scale)) return INDEXER_EINVAL;
+  if (p->visibility == INDEXER_VIS_POOLED && !pool_coef) return INDEXER_EINVAL;
+  size_t need = 0;
+  st = indexer_docs_workspace_bytes(p, doc_bounds, n_docs, &need);
+  if (st != INDEXER_OK) return st;
+  if (!workspace || !aligned(workspace, 256)) return INDEXER_EWORKSPACE;
+  if (workspace_bytes < need) return INDEXER_EWORKSPACE;
+  const bool fp8 = p->dtype == INDEXER_FP8_E4M3;
+  const size_t elem = fp8 ? 1 : 2;
+  int32_t width = 0;
+  st = indexer_out_width(p, &width);
+  if (st != INDEXER_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status word and counters start at zero once for all documents
+  if (cudaMemsetAsync(workspace, 0, 32, s) != cudaSuccess) return INDEXER_ECUDA;
+  for (int32_t d = 0; d < n_docs; ++d) {
+    DocPart part;
+    bool empty = false;
+    st = doc_part(p, doc_bounds, d, &part, &empty);
+    if (st != INDEXER_OK) return st;
+    if (empty) continue;
+    const int64_t r0 = part.r0;
+    const size_t q_row = static_cast<size_t>(p->H) * p->D * elem;
+    st = run_topk(&part.sub, q ? static_cast<const uint8_t*>(q) + r0 * q_row : nullptr,
+                  static_cast<const uint8_t*>(k) + part.key0 * static_cast<int64_t>(p->D) * elem,
+                  w ? w + r0 * p->H : nullptr, q_scale ? q_scale + r0 * p->H : nullptr,
+                  k_scale ? k_scale + part.key0 : nullptr, pool_coef, out_idx + r0 * width, out_len + r0,
+                  out_score ? out_score + r0 * width : nullptr, workspace, workspace_bytes, stream, false);
+    if (st != INDEXER_OK) return st;
+    if (launch_offset_indices(out_idx + r0 * width, part.sub.S * width, part.shift, s) != cudaSuccess)
+      return INDEXER_ECUDA;
+  }
+  return INDEXER_OK;
+}
+
+}  // extern "C"

@@ -88,6 +88,7 @@ cudaError_t launch_merge_splits(int64_t S, int64_t q_pos0, int splits, int ksel,
                                 const uint2* split_buf, const int32_t* split_cnt, const uint32_t* split_kth,
                                 const uint32_t* split_rth, uint2* gather, int64_t gather_stride, int32_t* out_idx, int32_t* out_len,
                                 float* out_score, cudaStream_t stream);
+cudaError_t launch_offset_indices(int32_t* idx, int64_t n, int32_t add, cudaStream_t stream);
 cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
                                 int32_t* shared, int32_t* left, int32_t* right, int32_t* counts,
                                 cudaStream_t stream);

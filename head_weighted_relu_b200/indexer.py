@@ -30,6 +30,7 @@ STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
 # every symbol include/hwr_indexer.h declares
 EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_topk_noalloc",
            "indexer_host_workspace_bytes", "indexer_topk_host",
+           "indexer_docs_workspace_bytes", "indexer_topk_docs",
            "indexer_pool_keys",
            "indexer_pair_overlap", "indexer_pair_regions", "indexer_read_status", "indexer_read_prune_counters",
            "indexer_status_string",
@@ -65,6 +66,8 @@ def _load():
     lib.indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.indexer_host_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
     lib.indexer_topk_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.indexer_docs_workspace_bytes.argtypes = [P, vp, i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.indexer_topk_docs.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_pool_keys.argtypes = [vp, i64, i32, vp, i32, vp, vp]
     lib.indexer_pair_overlap.argtypes = [vp, vp, i64, i32, vp, vp]
     lib.indexer_pair_regions.argtypes = [vp, vp, i64, i32, vp, vp, vp, vp, vp]
@@ -142,6 +145,31 @@ def indexer_topk_host(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, ou
     _check("indexer_topk_host", _lib.indexer_topk_host(
         ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
         _ptr(pool_coef), _ptr(out_idx), _ptr(out_len), _ptr(out_score), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def _bounds(doc_bounds):
+    import numpy as np
+    b = np.ascontiguousarray(np.asarray(doc_bounds, dtype=np.int64))
+    return b, ctypes.c_void_p(b.ctypes.data), len(b) - 1
+
+
+def indexer_docs_workspace_bytes(problem: Problem, doc_bounds) -> int:
+    b, ptr, n = _bounds(doc_bounds)
+    out = ctypes.c_size_t()
+    _check("indexer_docs_workspace_bytes",
+           _lib.indexer_docs_workspace_bytes(ctypes.byref(problem), ptr, n, ctypes.byref(out)))
+    return out.value
+
+
+def indexer_topk_docs(problem, q, k, w, q_scale, k_scale, pool_coef, doc_bounds, out_idx, out_len,
+                      out_score, workspace, stream=None):
+    """indexer_topk for a packed batch of documents: doc_bounds (host, n_docs + 1
+    token positions) splits the tokens; a query sees only its own document."""
+    b, ptr, n = _bounds(doc_bounds)
+    _check("indexer_topk_docs", _lib.indexer_topk_docs(
+        ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale), _ptr(pool_coef),
+        ptr, n, _ptr(out_idx), _ptr(out_len), _ptr(out_score), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

@@ -138,8 +138,12 @@ def generate(wl: Workload, device="cpu") -> dict:
         w = _randn((wl.S, wl.H), gen, device) * (1.0 / math.sqrt(wl.H))
         out["w"] = (w.abs() if wl.values == "corr" else w).to(torch.float32)
     if wl.visibility == POOLED:
-        c = torch.rand((wl.ratio, wl.D), generator=gen, device=device,
-                       dtype=torch.float32) * 0.5
+        if wl.values == "int":   # integer pooled keys: every score exact in FP32
+            c = torch.randint(0, 2, (wl.ratio, wl.D), generator=gen, device=device,
+                              dtype=torch.int32).to(torch.float32)
+        else:
+            c = torch.rand((wl.ratio, wl.D), generator=gen, device=device,
+                           dtype=torch.float32) * 0.5
         out["pool_coef"] = c.to(torch.bfloat16)
     return out
 

@@ -186,6 +186,33 @@ indexer_status indexer_topk_host(const indexer_problem* p, const void* q, const 
                                  int32_t* out_idx, int32_t* out_len, float* out_score,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* indexer_topk for a packed batch of documents ("Module 06 — DSA & KPool",
+ * §3 and "Ship it": no token of one document may reach another document's
+ * selection, and no pool may span a document boundary).  doc_bounds is a
+ * HOST array of n_docs + 1 token positions, strictly rising: document d is
+ * tokens [doc_bounds[d], doc_bounds[d+1]).  The query at global position g
+ * sees only keys of the document holding g:
+ *   TOKEN       tokens doc_start .. g;
+ *   COMPRESSED  compressed keys of its document (every bound a multiple of
+ *               the ratio; key j covers tokens ratio*j .. ratio*j+ratio-1);
+ *   POOLED      the document's own pools, formed from its tokens starting at
+ *               doc_start, then the document's incomplete tail.
+ * Every query position must lie inside [doc_bounds[0], doc_bounds[n_docs]),
+ * and doc_bounds[n_docs] within the keys.  Other arguments, output layout
+ * (global positions, -1 padding, lengths) and errors as indexer_topk; the
+ * workspace is indexer_docs_workspace_bytes bytes, and indexer_read_status
+ * covers all documents.  Each document runs as its own indexer call on
+ * `stream` (a few short documents are therefore cheaper batched into one
+ * problem without bounds). */
+indexer_status indexer_docs_workspace_bytes(const indexer_problem* p, const int64_t* doc_bounds,
+                                            int32_t n_docs, size_t* bytes);
+indexer_status indexer_topk_docs(const indexer_problem* p, const void* q, const void* k,
+                                 const float* w, const float* q_scale,
+                                 const float* k_scale, const void* pool_coef,
+                                 const int64_t* doc_bounds, int32_t n_docs,
+                                 int32_t* out_idx, int32_t* out_len, float* out_score,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Pool formation alone (the first step of POOLED):
  *   kp[p, d] = RNE_bf16( exact sum_{j<ratio} c[j, d] * k[ratio*p + j, d] )
  * for p < T_tokens / ratio; k [T_tokens, D] bf16, pool_coef [ratio, D] bf16,
