@@ -55,9 +55,17 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+        # wait (at most 3 s) for the first sample, taken before the timed
+        # region and left out of the summary, so that sampling is running
+        # when the region starts
+        if self.proc is not None:
+            import select
+            ready, _, _ = select.select([self.proc.stdout], [], [], 3.0)
+            if ready:
+                self.proc.stdout.readline()
         return self
 
     def __exit__(self, *a):
@@ -176,6 +184,21 @@ def run_reference(args, wl, world, rank):
     }))
 
 
+def planned_splits(wl, sms: int) -> int:
+    """Key-range splits the library plans for this shape (the host rule in
+    capi.cu): with fewer query blocks than half the SMs, SMs / blocks ranges of
+    at least 16 key tiles, at most 512.  A split shape adds the merge launch."""
+    qb = min(256 // wl.H, 32)
+    nb = -(-wl.S // qb)
+    if nb * 2 > sms:
+        return 1
+    g = wl.q_pos0 + wl.S - 1
+    n_keys = wl.T // wl.ratio if wl.visibility == W.POOLED else wl.T
+    nvis = min(g + 1 if wl.visibility == W.TOKEN else (g + 1) // wl.ratio, n_keys)
+    s = min(sms // nb, (nvis + 127) // 128 // 16, 512)
+    return s if s >= 2 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -260,6 +283,42 @@ def main():
         regions = {"ms_per_call": r_ms, "bytes_per_call": r_bytes, "gb_s": r_bytes / (r_ms * 1e-3) / 1e9}
         del outs, cnt
 
+    # decode-like shapes (few query blocks: split key ranges plus a merge) also
+    # time indexer_topk_witness, whose seed threshold shortens the per-range
+    # selection and the merge without changing the result.  Two seed sources:
+    # the same query rows' selection one decode step earlier (one key fewer;
+    # queries that change little between steps) and the row above's selection
+    # (on these i.i.d. synthetic queries it shares only chance keys).
+    splits = planned_splits(wl, torch.cuda.get_device_properties(dev).multi_processor_count)
+    witness = None
+    if splits > 1 and wl.visibility == W.TOKEN and wl.q_pos0 >= 1:
+        prev = I.make_problem(wl.S, wl.T - 1, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype, wl.q_pos0 - 1)
+        pb = I.allocate(prev, dev)
+        I.indexer_topk(prev, inp["q"], inp["k"], inp["w"], inp["q_scale"], inp["k_scale"], inp["pool_coef"],
+                       pb[0], pb[1], None, pb[3], stream)
+        seed_sets = {"prev_step": pb[0], "row_above": torch.roll(bufs[0], 1, 0).contiguous()}
+        wws = torch.empty(I.indexer_witness_workspace_bytes(prob, bufs[0].shape[1]), dtype=torch.uint8, device=dev)
+        w_idx, w_len = torch.empty_like(bufs[0]), torch.empty_like(bufs[1])
+        witness = {"api": "indexer_topk_witness", "ms_per_call_unseeded": ms_step, "seeds": {
+            "prev_step": "the same query rows' output over T - 1 keys",
+            "row_above": "output row t - 1 for query row t"}}
+        for name, sd in seed_sets.items():
+            def wstep():
+                I.indexer_topk_witness(prob, inp["q"], inp["k"], inp["w"], inp["q_scale"], inp["k_scale"],
+                                       inp["pool_coef"], sd, w_idx, w_len, None, wws, stream)
+            for _ in range(3):
+                wstep()
+            w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            w0.record(stream)
+            for _ in range(10):
+                wstep()
+            w1.record(stream)
+            torch.cuda.synchronize()
+            witness["ms_per_call_" + name] = w0.elapsed_time(w1) / 10
+            witness["identical_" + name] = bool(torch.equal(w_idx, bufs[0]) and torch.equal(w_len, bufs[1]))
+        witness["device_status"] = I.indexer_read_status(wws)
+        del pb, wws, w_idx, w_len, seed_sets
+
     pk = _peaks()
     tensor_peak = pk["bf16"] * (2.0 if wl.dtype == "fp8" else 1.0)
     kern_ms = statistics.mean(per)
@@ -312,7 +371,8 @@ def main():
     except Exception:
         traffic = None
 
-    launches_per_step = 1 + (1 if wl.visibility == W.POOLED else 0) + (1 if wl.pair_overlap else 0)
+    launches_per_step = (1 + (1 if splits > 1 else 0) + (1 if wl.visibility == W.POOLED else 0)
+                         + (1 if wl.pair_overlap else 0))
     if rank == 0:
         out = {
             "metric": METRIC, "value": value, "unit": "Gpairs/s", "n_gpus": world,
@@ -337,6 +397,7 @@ def main():
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "pair_regions": regions,
+            "witness": witness,
             "device_status": status,
             "cpu_baseline": base,
         }

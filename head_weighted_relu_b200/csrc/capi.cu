@@ -216,12 +216,26 @@ indexer_status indexer_workspace_bytes(const indexer_problem* p, size_t* bytes) 
 namespace hwr {
 namespace {
 
+// Seeds of indexer_topk_witness: [S, n] key rows per query, and the scratch
+// after the indexer's own workspace.
+struct Seeds {
+  const int32_t* idx;
+  int64_t n;
+  uint32_t* lowered;  // [S, n]
+  uint32_t* thr;      // [S]
+};
+
+size_t witness_extra_bytes(int64_t S, int64_t n_seeds) {
+  return align256(static_cast<size_t>(S) * n_seeds * sizeof(uint32_t)) + align256(static_cast<size_t>(S) * 4);
+}
+
 // indexer_topk; reset_status = false leaves the device status word as it is
 // (the host pipeline resets it once and runs one call per chunk of rows).
+// With seeds, every query starts from the seed threshold.
 indexer_status run_topk(const indexer_problem* p, const void* q, const void* k, const float* w,
                         const float* q_scale, const float* k_scale, const void* pool_coef, int32_t* out_idx,
                         int32_t* out_len, float* out_score, void* workspace, size_t workspace_bytes,
-                        void* stream_, bool reset_status) {
+                        void* stream_, bool reset_status, const Seeds* seeds = nullptr) {
   Plan pl;
   indexer_status st = make_plan(p, true, &pl);
   if (st != INDEXER_OK) return st;
@@ -299,6 +313,31 @@ indexer_status run_topk(const indexer_problem* p, const void* q, const void* k, 
   sp.split_cnt = split_cnt;
   sp.split_kth = split_kth;
   sp.split_rth = split_rth;
+  sp.seed_thr = nullptr;
+  if (seeds) {
+    WitnessParams wp;
+    wp.S = p->S;
+    wp.n_keys = pl.n_keys;
+    wp.q_pos0 = p->q_pos0;
+    wp.H = p->H;
+    wp.ranged = pl.ranged;
+    wp.ratio = sp.ratio;
+    wp.seed_div = pl.out_ratio;
+    wp.ksel = pl.ksel;
+    wp.fp8 = fp8 ? 1 : 0;
+    wp.n_seeds = seeds->n;
+    wp.seed_stride = seeds->n;
+    wp.q = q;
+    wp.w = w;
+    wp.q_scale = q_scale;
+    wp.keys = keys;
+    wp.k_scale = k_scale;
+    wp.seeds = seeds->idx;
+    wp.lowered = seeds->lowered;
+    wp.thr = seeds->thr;
+    if (launch_witness(wp, p->D, stream) != cudaSuccess) return INDEXER_ECUDA;
+    sp.seed_thr = seeds->thr;
+  }
   if (pl.prune && launch_prune_setup(q, w, q_scale, fp8, p->S, p->H, p->D, keys, pl.n_keys, pq, knorm,
                                      stream) != cudaSuccess)
     return INDEXER_ECUDA;
@@ -312,7 +351,7 @@ indexer_status run_topk(const indexer_problem* p, const void* q, const void* k, 
   if (pl.splits > 1 &&
       launch_merge_splits(p->S, p->q_pos0, pl.splits, pl.ksel, pl.width, pl.out_ratio, split_buf, split_cnt,
                           split_kth, split_rth, split_gather, pl.gather_stride, out_idx, out_len, out_score,
-                          stream) != cudaSuccess)
+                          MergeCheck{seeds ? 1 : 0, pl.ranged, sp.ratio, pl.n_keys, status}, stream) != cudaSuccess)
     return INDEXER_ECUDA;
   return INDEXER_OK;
 }
@@ -328,6 +367,34 @@ indexer_status indexer_topk(const indexer_problem* p, const void* q, const void*
                             void* stream) {
   return hwr::run_topk(p, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len, out_score, workspace,
                        workspace_bytes, stream, true);
+}
+
+indexer_status indexer_witness_workspace_bytes(const indexer_problem* p, int64_t n_seeds, size_t* bytes) {
+  Plan pl;
+  const indexer_status st = make_plan(p, true, &pl);
+  if (st != INDEXER_OK) return st;
+  if (!bytes || n_seeds < 0 || n_seeds > (int64_t(1) << 20)) return INDEXER_EINVAL;
+  *bytes = pl.ws_bytes + hwr::witness_extra_bytes(p->S, n_seeds);
+  return INDEXER_OK;
+}
+
+indexer_status indexer_topk_witness(const indexer_problem* p, const void* q, const void* k, const float* w,
+                                    const float* q_scale, const float* k_scale, const void* pool_coef,
+                                    const int32_t* seeds, int64_t n_seeds, int32_t* out_idx, int32_t* out_len,
+                                    float* out_score, void* workspace, size_t workspace_bytes, void* stream) {
+  Plan pl;
+  indexer_status st = make_plan(p, true, &pl);
+  if (st != INDEXER_OK) return st;
+  if (n_seeds < 0 || n_seeds > (int64_t(1) << 20) || (p->S > 0 && n_seeds > 0 && !seeds))
+    return INDEXER_EINVAL;
+  if (p->H > 64 || (p->D != 64 && p->D != 128)) return INDEXER_EUNSUPPORTED;
+  if (!workspace || workspace_bytes < pl.ws_bytes + hwr::witness_extra_bytes(p->S, n_seeds))
+    return INDEXER_EWORKSPACE;
+  uint8_t* extra = static_cast<uint8_t*>(workspace) + pl.ws_bytes;
+  const hwr::Seeds sd{seeds, n_seeds, reinterpret_cast<uint32_t*>(extra),
+                      reinterpret_cast<uint32_t*>(extra + align256(static_cast<size_t>(p->S) * n_seeds * 4))};
+  return hwr::run_topk(p, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len, out_score, workspace,
+                       workspace_bytes, stream, true, &sd);
 }
 
 indexer_status indexer_pool_keys(const void* k, int64_t T_tokens, int32_t D, const void* pool_coef,

@@ -11,6 +11,7 @@ namespace hwr {
 // Device status bits kept in the first word of the workspace.
 constexpr uint32_t kStatusWaitTimeout = 1u;
 constexpr uint32_t kStatusOverflow = 2u;
+constexpr uint32_t kStatusWitness = 4u;  // a seed threshold left a query fewer than min(K, visible) keys
 
 // Heads the pruning certificate keeps exactly (the first kPruneR of each query).
 constexpr int kPruneR = 16;
@@ -45,6 +46,7 @@ struct ScoreParams {
   uint32_t* split_kth;   // splits > 1: [S][splits] ordered score of each full split's K-th entry, else 0
   uint32_t* split_rth;   // splits > 1: [S][splits] ordered score of each split's r-th entry, r = ceil(K / splits)
                          // (0 when it has fewer than r)
+  const uint32_t* seed_thr;  // [S] ordered-score threshold every query starts from, or null (0 for all)
 };
 
 // Per-variant launch facts, filled by the kernel's translation unit.
@@ -84,10 +86,44 @@ cudaError_t launch_prune_setup(const void* q, const float* w, const float* q_sca
 // per-split offsets in shared memory).
 constexpr int kMaxSplits = 512;
 
+// Visibility facts the merge needs to check a seeded run (seeded = 0: none).
+struct MergeCheck {
+  int32_t seeded;
+  int32_t ranged;
+  int32_t ratio;
+  int64_t n_keys;
+  uint32_t* status;
+};
+
 cudaError_t launch_merge_splits(int64_t S, int64_t q_pos0, int splits, int ksel, int width, int out_ratio,
                                 const uint2* split_buf, const int32_t* split_cnt, const uint32_t* split_kth,
                                 const uint32_t* split_rth, uint2* gather, int64_t gather_stride, int32_t* out_idx, int32_t* out_len,
-                                float* out_score, cudaStream_t stream);
+                                float* out_score, const MergeCheck& check, cudaStream_t stream);
+
+// Seed thresholds (witness.cu): thr[t] = the ksel-th largest lowered exact
+// score over the distinct visible key rows that row t of `seeds` names.
+struct WitnessParams {
+  int64_t S;
+  int64_t n_keys;       // rows of the scored key matrix
+  int64_t q_pos0;
+  int32_t H;
+  int32_t ranged;       // visibility as in ScoreParams
+  int32_t ratio;
+  int32_t seed_div;     // seeds name key row e / seed_div (POOLED: token positions -> pools)
+  int32_t ksel;
+  int32_t fp8;
+  int64_t n_seeds;      // seeds per row
+  int64_t seed_stride;  // row stride of seeds
+  const void* q;        // [S, H, D] (bf16 values or e4m3 codes)
+  const float* w;       // [S, H]
+  const float* q_scale; // [S, H] (FP8)
+  const void* keys;     // [n_keys, D]: the scored key matrix (pools for POOLED)
+  const float* k_scale; // [n_keys] (FP8)
+  const int32_t* seeds; // [S, seed_stride]; -1 or any other invalid entry is ignored
+  uint32_t* lowered;    // [S, n_seeds] scratch
+  uint32_t* thr;        // [S] result
+};
+cudaError_t launch_witness(const WitnessParams& wp, int D, cudaStream_t stream);
 cudaError_t launch_offset_indices(int32_t* idx, int64_t n, int32_t add, cudaStream_t stream);
 cudaError_t launch_pair_regions(const int32_t* idx, const int32_t* len, int64_t n_pairs, int width,
                                 int32_t* shared, int32_t* left, int32_t* right, int32_t* counts,

@@ -205,6 +205,7 @@ struct MergeParams {
   int32_t* out_idx;
   int32_t* out_len;
   float* out_score;
+  MergeCheck check;
 };
 
 // One CTA of 128 threads (one warpgroup) per query row.
@@ -212,6 +213,8 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
   __shared__ uint32_t hist[kHistBins];
   __shared__ WgState<1> st;
   __shared__ uint32_t bound_s[2];
+  __shared__ int32_t off_s[kMaxSplits + 1];  // start of each range's list in the gathered row
+  __shared__ int32_t wsum_s[kBM / 32];
   const int etid = threadIdx.x;
   const int lane = etid & 31;
   constexpr int bar_id = 1;
@@ -238,14 +241,54 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
     }
     named_bar(bar_id, kBM);
     const uint32_t bound = max(bound_s[0], bound_s[1]);
-    // concatenate the lists in range order, keeping entries >= bound
+    // offsets of the lists: thread etid owns ranges 4 etid .. 4 etid + 3
+    // (splits <= 512 = 4 x 128), exclusive scan over the group
+    int32_t c4[4], local = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sp = 4 * etid + u;
+      c4[u] = sp < mp.splits ? cnt[sp] : 0;
+      local += c4[u];
+    }
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t v = __shfl_up_sync(kFullMask, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum_s[etid >> 5] = incl;
+    named_bar(bar_id, kBM);
+    int32_t run = incl - local;
+    for (int w2 = 0; w2 < (etid >> 5); ++w2) run += wsum_s[w2];
+    const int32_t total = wsum_s[0] + wsum_s[1] + wsum_s[2] + wsum_s[3];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sp = 4 * etid + u;
+      if (sp < mp.splits) off_s[sp] = run;
+      run += c4[u];
+    }
+    named_bar(bar_id, kBM);
+    // concatenate the lists in range order (key order).  Short lists (a seed
+    // threshold leaves about K entries in all), or lists with no bound to
+    // filter by, are copied whole, one warp per range, with no barrier
+    // between ranges; long ones keep only entries >= bound, range by range
     uint2* buf = mp.gather + static_cast<size_t>(t) * mp.gather_stride;
-    const Cut keep_from{bound, 0xFFFFFFFFu};  // keeps ordered scores >= bound
     int n = 0;
-    for (int sp = 0; sp < mp.splits; ++sp) {
-      const uint2* src = mp.split_buf + (static_cast<size_t>(t) * mp.splits + sp) * mp.ksel;
-      n += m_compact(src, cnt[sp], keep_from, bound == 0u, &st.cwc[0][0], etid, bar_id,
-                     [&](int pos, uint2 e) { buf[n + pos] = e; });
+    if (total <= kRegCap || bound == 0u) {
+      const int wq = etid >> 5;
+      for (int sp = wq; sp < mp.splits; sp += kBM / 32) {
+        const uint2* src = mp.split_buf + (static_cast<size_t>(t) * mp.splits + sp) * mp.ksel;
+        const int c = cnt[sp], o = off_s[sp];
+        for (int i = lane; i < c; i += 32) buf[o + i] = src[i];
+      }
+      n = total;
+    } else {
+      const Cut keep_from{bound, 0xFFFFFFFFu};  // keeps ordered scores >= bound
+      for (int sp = 0; sp < mp.splits; ++sp) {
+        const uint2* src = mp.split_buf + (static_cast<size_t>(t) * mp.splits + sp) * mp.ksel;
+        n += m_compact(src, cnt[sp], keep_from, bound == 0u, &st.cwc[0][0], etid, bar_id,
+                       [&](int pos, uint2 e) { buf[n + pos] = e; });
+      }
     }
     named_bar(bar_id, kBM);  // the gathered list is visible to the group
 
@@ -288,7 +331,16 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
       orow[i] = -1;
       if (srow) srow[i] = __uint_as_float(0x7FC00000u);
     }
-    if (etid == 0) mp.out_len[t] = len;
+    if (etid == 0) {
+      mp.out_len[t] = len;
+      if (mp.check.seeded) {
+        // with a seed threshold at least min(K, visible) keys must pass it
+        const int64_t g = mp.q_pos0 + t;
+        int64_t nvis = mp.check.ranged ? (g + 1) / mp.check.ratio : g + 1;
+        if (nvis > mp.check.n_keys) nvis = mp.check.n_keys;
+        if (kept < min(static_cast<int64_t>(mp.ksel), nvis)) atomicOr(mp.check.status, kStatusWitness);
+      }
+    }
     named_bar(bar_id, kBM);  // the selection scratch is reused by the next row
   }
 }
@@ -296,14 +348,14 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
 cudaError_t launch_merge_splits(int64_t S, int64_t q_pos0, int splits, int ksel, int width, int out_ratio,
                                 const uint2* split_buf, const int32_t* split_cnt, const uint32_t* split_kth,
                                 const uint32_t* split_rth, uint2* gather, int64_t gather_stride, int32_t* out_idx, int32_t* out_len,
-                                float* out_score, cudaStream_t stream) {
+                                float* out_score, const MergeCheck& check, cudaStream_t stream) {
   if (S == 0) return cudaSuccess;
   if (splits > kMaxSplits) return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const MergeParams mp{S, q_pos0, splits, ksel, width, out_ratio, split_buf, split_cnt, split_kth, split_rth,
-                       gather, gather_stride, out_idx, out_len, out_score};
+                       gather, gather_stride, out_idx, out_len, out_score, check};
   int64_t blocks = S < static_cast<int64_t>(sms) * 8 ? S : static_cast<int64_t>(sms) * 8;
   merge_splits_kernel<<<static_cast<unsigned>(blocks), kBM, 0, stream>>>(mp);
   return cudaGetLastError();

@@ -16,6 +16,16 @@
 // codes the MMA multiplies, w already carries the q scale, and the key scale
 // multiplies U after the sum exactly as it multiplies the score.
 //
+// The residual allowance is the smaller of two bounds of
+//   R = sum_h [x_h . k]_+,   x_h = w_h d_h   (both signs of w_h),
+// the per-head one E_P |k| = sum_h |x_h| |k|, and the same page's joint one
+// (技术新颖性, second point), which uses how the residuals align:
+//   R = 1/2 ((sum_h x_h) . k + sum_h |x_h . k|)
+//     <= 1/2 (|sum_h x_h| + sqrt(sum_{h,l} |x_h . x_l|)) |k| = E_joint |k|,
+// since sum_h |x_h . k| = (sum_h s_h x_h) . k for signs s_h, and
+// |sum_h s_h x_h|^2 <= sum_{h,l} |x_h . x_l|.  E_joint <= E_P always; for
+// nearly orthogonal residuals it is about sqrt(#heads) times smaller.
+//
 // The margin covers the MMA's accumulation error and the FP32 rounding of
 // both the score and U: 2^-11 * |k| * sum_h |w_h| |q_h|.
 #include <cuda_bf16.h>
@@ -45,18 +55,18 @@ __device__ __forceinline__ float warp_sum_f32(float v) {
 // FP32 computation approximated (relative 2^-18 covers a few roundings).
 __device__ __forceinline__ float round_up_pos(float x) { return x * (1.0f + 0x1p-18f) + 0x1p-100f; }
 
-// One warp per query row t: out[t] = {wt[0..r), Ceff}.  Requires D % 32 == 0
-// and D <= 128 (four values per lane), H <= 64.
-__global__ void prune_prep_kernel(const void* __restrict__ q, const float* __restrict__ w,
-                                  const float* __restrict__ q_scale, bool fp8, int64_t S, int H, int D,
-                                  float* __restrict__ out) {
+// One warp (the whole block) per query row t: out[t] = {wt[0..r), Ceff,
+// sum |w||q|}.  Requires D % 32 == 0 and D <= 128 (four values per lane),
+// H <= 64.  The omitted heads' residuals x_h are kept in shared memory for the
+// joint bound's Gram sum.
+__global__ void __launch_bounds__(32) prune_prep_kernel(const void* __restrict__ q, const float* __restrict__ w,
+                                                        const float* __restrict__ q_scale, bool fp8, int64_t S,
+                                                        int H, int D, float* __restrict__ out) {
   const int lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
-  __shared__ float wt_s[8][kPruneR];
-  float* wt = wt_s[threadIdx.x >> 5];
+  __shared__ float wt[kPruneR];
+  __shared__ float xs[64 - kPruneR][128];  // x_h = w_h d_h, head h - kPruneR, dims lane + 32 m
   const int per = D / 32;  // values per lane
-  for (int64_t t = blockIdx.x * static_cast<int64_t>(warps) + (threadIdx.x >> 5); t < S;
-       t += static_cast<int64_t>(gridDim.x) * warps) {
+  for (int64_t t = blockIdx.x; t < S; t += gridDim.x) {
     const size_t qbase = static_cast<size_t>(t) * H * D;
     // kept heads in registers: head j, dims lane + 32 m
     float kept[kPruneR][4];
@@ -78,6 +88,8 @@ __global__ void prune_prep_kernel(const void* __restrict__ q, const float* __res
     }
     __syncwarp();
     float C = 0.f;
+    float xsum[4] = {0.f, 0.f, 0.f, 0.f};  // sum_h x_h (this lane's dims)
+    float G = 0.f;                         // sum_{h,l} |x_h . x_l|
     for (int h = kPruneR; h < H; ++h) {
       float v[4];
       float ss = 0.f;
@@ -131,10 +143,45 @@ __global__ void prune_prep_kernel(const void* __restrict__ q, const float* __res
         if (lane == 0) wt[best] += wh * beta;
       }
       C += fabsf(wh) * nd;
+      // x_h = w_h d_h (the FP32 residual; the joint bound's slack below covers
+      // its rounding), its Gram terms with the earlier residuals, and the sum
+      float x[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float d = v[m];
+#pragma unroll
+        for (int j = 0; j < kPruneR; ++j)
+          if (j == best) d = fmaf(-beta, kept[j][m], v[m]);
+        x[m] = m < per ? wh * d : 0.f;
+        xsum[m] += x[m];
+      }
+      float xx = 0.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) xx = fmaf(x[m], x[m], xx);
+      G += warp_sum_f32(xx);
+      for (int l = 0; l < h - kPruneR; ++l) {
+        float dd = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          if (m < per) dd = fmaf(x[m], xs[l][lane + 32 * m], dd);
+        G += 2.f * fabsf(warp_sum_f32(dd));
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (m < per) xs[h - kPruneR][lane + 32 * m] = x[m];
       __syncwarp();
     }
-    __syncwarp();
-    const float ceff = round_up_pos(round_up_pos(C) + 0x1p-11f * wsum);
+    float sx = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) sx = fmaf(xsum[m], xsum[m], sx);
+    sx = warp_sum_f32(sx);
+    // FP32 slack of the joint bound: the Gram sum and |sum x| carry relative
+    // errors of about D * 2^-24 of (sum |x_h|)^2 and sum |x_h|, and x_h
+    // itself differs from w_h (q_h - beta q_j) by 2^-20-relative amounts;
+    // 2^-7 * C (about 0.8% of the per-head bound) covers all of them
+    const float joint = round_up_pos(0.5f * (sqrtf(sx) + sqrtf(G))) + 0x1p-7f * C;
+    const float resid = fminf(round_up_pos(C), joint);
+    const float ceff = round_up_pos(resid + 0x1p-11f * wsum);
     float* o = out + static_cast<size_t>(t) * (kPruneR + 2);
     if (lane < kPruneR) o[lane] = wt[lane];
     if (lane == 0) {
@@ -169,9 +216,9 @@ cudaError_t launch_prune_setup(const void* q, const float* w, const float* q_sca
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int threads = 256;  // 8 warps
   if (S > 0) {
-    int64_t blocks = (S + 7) / 8;
-    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
-    prune_prep_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(q, w, q_scale, fp8, S, H, D, pq);
+    int64_t blocks = S;  // one warp per query row
+    if (blocks > static_cast<int64_t>(sms) * 32) blocks = static_cast<int64_t>(sms) * 32;
+    prune_prep_kernel<<<static_cast<unsigned>(blocks), 32, 0, stream>>>(q, w, q_scale, fp8, S, H, D, pq);
   }
   if (n_keys > 0) {
     int64_t blocks = (n_keys + 7) / 8;

@@ -816,7 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t t = tq0 + etid;
         st->nvis[etid] = t < p.S ? n_visible(p, p.q_pos0 + t) : 0;
         st->cnt[par][etid] = 0;
-        st->thr[etid] = 0u;
+        // a seed threshold, when given, is a lower bound of the K-th score
+        st->thr[etid] = (p.seed_thr != nullptr && t < p.S) ? p.seed_thr[t] : 0u;
       }
       named_bar(bar_id, kBM);
 
@@ -1095,7 +1096,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               orow[i] = -1;
               if (srow) srow[i] = __uint_as_float(0x7FC00000u);
             }
-            if (etid == 0) p.out_len[t] = len;
+            if (etid == 0) {
+              p.out_len[t] = len;
+              // with a seed threshold at least min(K, visible) keys must pass it
+              if (p.seed_thr != nullptr && kept < min(p.ksel, st->nvis[qi])) atomicOr(p.status, kStatusWitness);
+            }
           }
           named_bar(bar_id, kBM);
         }

@@ -31,6 +31,7 @@ STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
 EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_topk_noalloc",
            "indexer_host_workspace_bytes", "indexer_topk_host",
            "indexer_docs_workspace_bytes", "indexer_topk_docs",
+           "indexer_witness_workspace_bytes", "indexer_topk_witness",
            "indexer_pool_keys",
            "indexer_pair_overlap", "indexer_pair_regions", "indexer_read_status", "indexer_read_prune_counters",
            "indexer_status_string",
@@ -68,6 +69,8 @@ def _load():
     lib.indexer_topk_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_docs_workspace_bytes.argtypes = [P, vp, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.indexer_topk_docs.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.indexer_witness_workspace_bytes.argtypes = [P, i64, ctypes.POINTER(ctypes.c_size_t)]
+    lib.indexer_topk_witness.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_pool_keys.argtypes = [vp, i64, i32, vp, i32, vp, vp]
     lib.indexer_pair_overlap.argtypes = [vp, vp, i64, i32, vp, vp]
     lib.indexer_pair_regions.argtypes = [vp, vp, i64, i32, vp, vp, vp, vp, vp]
@@ -126,6 +129,27 @@ def indexer_topk(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len
     _check("indexer_topk", _lib.indexer_topk(
         ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
         _ptr(pool_coef), _ptr(out_idx), _ptr(out_len), _ptr(out_score), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def indexer_witness_workspace_bytes(problem: Problem, n_seeds: int) -> int:
+    n = ctypes.c_size_t()
+    _check("indexer_witness_workspace_bytes",
+           _lib.indexer_witness_workspace_bytes(ctypes.byref(problem), ctypes.c_int64(n_seeds), ctypes.byref(n)))
+    return n.value
+
+
+def indexer_topk_witness(problem, q, k, w, q_scale, k_scale, pool_coef, seeds, out_idx, out_len, out_score,
+                         workspace, stream=None):
+    """indexer_topk starting from a seed threshold: seeds is a [S, n] int32
+    device tensor of key indices per query (e.g. the previous decode step's
+    out_idx), -1 or invisible entries ignored.  Same result as indexer_topk."""
+    if seeds.dtype != torch.int32 or seeds.dim() != 2 or not seeds.is_contiguous():
+        raise ValueError("seeds must be a contiguous [S, n] int32 tensor")
+    _check("indexer_topk_witness", _lib.indexer_topk_witness(
+        ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
+        _ptr(pool_coef), _ptr(seeds), ctypes.c_int64(seeds.shape[1]), _ptr(out_idx), _ptr(out_len),
+        _ptr(out_score), _ptr(workspace),
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
 
 

@@ -186,6 +186,46 @@ indexer_status indexer_topk_host(const indexer_problem* p, const void* q, const 
                                  int32_t* out_idx, int32_t* out_len, float* out_score,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* indexer_topk starting from a seed threshold ("DoSA: Dots Sparse
+ * Attention", 核心方法 / core method, first step: score at least K visible
+ * seed keys exactly and take their K-th score as a lower bound tau of the
+ * query's K-th score; 实验结果 / results: in decode the threshold comes from
+ * keys selected at recent steps and cuts the selection work).
+ *   seeds  [S, n_seeds] int32 DEVICE array: for each query row, key indices
+ *          in the numbering of out_idx -- token positions for TOKEN and
+ *          POOLED (a position names the pool that holds it), compressed-key
+ *          indices for COMPRESSED.  The previous decode step's out_idx row is
+ *          a typical seed row.  Entries that are negative or not visible to
+ *          the query are ignored, and so is any entry naming a key at or below
+ *          the largest key named earlier in its row (so rows in ascending
+ *          order are used whole, and no key counts twice).
+ * Each row's remaining seeds are scored exactly in FP32 on CUDA cores,
+ * lowered by a margin that covers the difference to the tensor-core scores
+ * (eps |k| sum_h |w_h||q_h| with eps = 2^-12 for BF16 and 2^-9 for FP8, times
+ * the key scale for FP8), and their K-th
+ * largest (K/ratio-th for POOLED) becomes the query's starting threshold; with
+ * fewer seeds than that the query starts from no threshold.  Keys below the
+ * threshold never become candidates, which shortens the selection and, with
+ * split key ranges, the merge; the result is identical to indexer_topk's.
+ * A run in which some query kept fewer than min(K, visible) keys sets bit 2
+ * of the status word (never expected: the margin was too small).  That is the
+ * only way a too-small margin can show: a threshold above the true K-th score
+ * leaves fewer than K keys at or above it, so no wrong row is full-length.
+ *   workspace: indexer_witness_workspace_bytes bytes (the indexer's own
+ * workspace, then the seed scores [S, n_seeds] and thresholds [S]).
+ * n_seeds may be 0 (then nothing is seeded); INDEXER_EINVAL for n_seeds < 0
+ * or > 2^20 or a null `seeds` with S, n_seeds > 0; INDEXER_EUNSUPPORTED for
+ * H > 64 or D other than 64 and 128.  Scoring the seeds costs H*D multiply-
+ * adds per seed on CUDA cores: meant for decode shapes (few rows). */
+indexer_status indexer_witness_workspace_bytes(const indexer_problem* p, int64_t n_seeds,
+                                               size_t* bytes);
+indexer_status indexer_topk_witness(const indexer_problem* p, const void* q, const void* k,
+                                    const float* w, const float* q_scale,
+                                    const float* k_scale, const void* pool_coef,
+                                    const int32_t* seeds, int64_t n_seeds,
+                                    int32_t* out_idx, int32_t* out_len, float* out_score,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* indexer_topk for a packed batch of documents ("Module 06 — DSA & KPool",
  * §3 and "Ship it": no token of one document may reach another document's
  * selection, and no pool may span a document boundary).  doc_bounds is a
@@ -253,7 +293,9 @@ indexer_status indexer_pair_regions(const int32_t* idx, const int32_t* len,
 /* Synchronises `stream`, then reads the device status word that indexer_topk
  * keeps in `workspace` (0 = no fault).  Bit 0: a pipeline wait in the kernel
  * gave up after its time limit (the result is not valid); bit 1: a candidate
- * buffer would have overflowed (never expected; the result is not valid).
+ * buffer would have overflowed (never expected; the result is not valid);
+ * bit 2: a seed threshold of indexer_topk_witness was above some query's
+ * K-th score (never expected; that row may be short).
  * Also clears the word.  Host pointer `flags`. */
 indexer_status indexer_read_status(void* workspace, int32_t* flags, void* stream);
 
