@@ -57,20 +57,39 @@ __device__ __forceinline__ float round_up_pos(float x) { return x * (1.0f + 0x1p
 
 // One warp (the whole block) per query row t: out[t] = {wt[0..r), Ceff,
 // sum |w||q|}.  Requires D % 32 == 0 and D <= 128 (four values per lane),
-// H <= 64.  The omitted heads' residuals x_h are kept in shared memory for the
-// joint bound's Gram sum.
+// H <= 64.  Dot products between heads run one per lane over rows staged in
+// shared memory (a padded row stride keeps lanes on different rows off each
+// other's banks), so a query's set-up is a few long independent chains
+// rather than one warp reduction per pair -- it is on the critical path of
+// decode-like shapes, which have a handful of query rows.
+constexpr int kRow = 129;  // padded row stride (floats)
+
+// sum_d a[d] b[d] over D dims of two shared-memory rows, four chains.
+__device__ __forceinline__ float row_dot(const float* a, const float* b, int D) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  for (int d = 0; d < D; d += 4) {
+    s0 = fmaf(a[d], b[d], s0);
+    s1 = fmaf(a[d + 1], b[d + 1], s1);
+    s2 = fmaf(a[d + 2], b[d + 2], s2);
+    s3 = fmaf(a[d + 3], b[d + 3], s3);
+  }
+  return (s0 + s1) + (s2 + s3);
+}
+
 __global__ void __launch_bounds__(32) prune_prep_kernel(const void* __restrict__ q, const float* __restrict__ w,
                                                         const float* __restrict__ q_scale, bool fp8, int64_t S,
                                                         int H, int D, float* __restrict__ out) {
   const int lane = threadIdx.x & 31;
   __shared__ float wt[kPruneR];
-  __shared__ float xs[64 - kPruneR][128];  // x_h = w_h d_h, head h - kPruneR, dims lane + 32 m
+  __shared__ float nk_s[kPruneR];
+  __shared__ float qk[kPruneR][kRow];        // kept heads
+  __shared__ float qv[kRow];                 // the omitted head being folded
+  __shared__ float xs[64 - kPruneR][kRow];   // x_h = w_h d_h, row h - kPruneR
   const int per = D / 32;  // values per lane
   for (int64_t t = blockIdx.x; t < S; t += gridDim.x) {
     const size_t qbase = static_cast<size_t>(t) * H * D;
-    // kept heads in registers: head j, dims lane + 32 m
+    // kept heads in registers (head j, dims lane + 32 m) and in shared memory
     float kept[kPruneR][4];
-    float nkept[kPruneR];
     float wsum = 0.f;  // sum_h |w_h| |q_h|, rounded up
 #pragma unroll
     for (int j = 0; j < kPruneR; ++j) {
@@ -79,17 +98,21 @@ __global__ void __launch_bounds__(32) prune_prep_kernel(const void* __restrict__
       for (int m = 0; m < 4; ++m) {
         kept[j][m] = m < per ? load_q_elem(q, fp8, qbase + static_cast<size_t>(j) * D + lane + 32 * m) : 0.f;
         ss = fmaf(kept[j][m], kept[j][m], ss);
+        if (m < per) qk[j][lane + 32 * m] = kept[j][m];
       }
-      nkept[j] = round_up_pos(sqrtf(warp_sum_f32(ss)));
+      const float nj = round_up_pos(sqrtf(warp_sum_f32(ss)));
       float wj = w[t * H + j];
       if (fp8) wj *= q_scale[t * H + j];
-      if (lane == 0) wt[j] = wj;
-      wsum += fabsf(wj) * nkept[j];
+      if (lane == 0) {
+        wt[j] = wj;
+        nk_s[j] = nj;
+      }
+      wsum += fabsf(wj) * nj;
     }
     __syncwarp();
     float C = 0.f;
     float xsum[4] = {0.f, 0.f, 0.f, 0.f};  // sum_h x_h (this lane's dims)
-    float G = 0.f;                         // sum_{h,l} |x_h . x_l|
+    float gdiag = 0.f;                     // this lane's part of sum_h |x_h|^2
     for (int h = kPruneR; h < H; ++h) {
       float v[4];
       float ss = 0.f;
@@ -97,80 +120,71 @@ __global__ void __launch_bounds__(32) prune_prep_kernel(const void* __restrict__
       for (int m = 0; m < 4; ++m) {
         v[m] = m < per ? load_q_elem(q, fp8, qbase + static_cast<size_t>(h) * D + lane + 32 * m) : 0.f;
         ss = fmaf(v[m], v[m], ss);
+        if (m < per) qv[lane + 32 * m] = v[m];
       }
+      __syncwarp();
       const float nh = round_up_pos(sqrtf(warp_sum_f32(ss)));
       float wh = w[t * H + h];
       if (fp8) wh *= q_scale[t * H + h];
       wsum += fabsf(wh) * nh;
-      // anchor: the kept head with the largest positive projection
-      int best = -1;
-      float best_proj = 0.f, best_dot = 0.f;
+      // anchor: the kept head with the largest positive projection (lane j
+      // computes q_h . q_j; ties go to the lower j)
+      float dd = 0.f, proj = -1.f;
+      if (lane < kPruneR) {
+        dd = row_dot(qv, qk[lane], D);
+        proj = (dd > 0.f && nk_s[lane] > 0.f) ? dd / nk_s[lane] : -1.f;
+      }
+      int best = lane < kPruneR ? lane : kPruneR;
 #pragma unroll
-      for (int j = 0; j < kPruneR; ++j) {
-        float dd = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) dd = fmaf(v[m], kept[j][m], dd);
-        dd = warp_sum_f32(dd);
-        const float proj = nkept[j] > 0.f ? dd / nkept[j] : 0.f;
-        if (dd > 0.f && proj > best_proj) {
-          best = j;
-          best_proj = proj;
-          best_dot = dd;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float p2 = __shfl_xor_sync(kFullMask, proj, o);
+        const int b2 = __shfl_xor_sync(kFullMask, best, o);
+        if (p2 > proj || (p2 == proj && b2 < best)) {
+          proj = p2;
+          best = b2;
         }
       }
+      const float best_dot = __shfl_sync(kFullMask, dd, best & 31);
+      if (proj <= 0.f) best = -1;
       float beta = 0.f, nd = nh;
+      float d[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) d[m] = v[m];
       if (best >= 0) {
         // any beta >= 0 gives a valid bound once |d| is measured for that beta
-        float nj2 = 0.f;
-#pragma unroll
-        for (int j = 0; j < kPruneR; ++j)
-          if (j == best) nj2 = nkept[j] * nkept[j];
+        const float nj = nk_s[best];
+        const float nj2 = nj * nj;
         beta = best_dot / nj2;
         float ds = 0.f;
 #pragma unroll
-        for (int j = 0; j < kPruneR; ++j)
-          if (j == best) {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const float d = fmaf(-beta, kept[j][m], v[m]);
-              ds = fmaf(d, d, ds);
-            }
-          }
+        for (int m = 0; m < 4; ++m) {
+          d[m] = m < per ? fmaf(-beta, qk[best][lane + 32 * m], v[m]) : 0.f;
+          ds = fmaf(d[m], d[m], ds);
+        }
         nd = round_up_pos(sqrtf(warp_sum_f32(ds)));
         // the FP32 residual d differs from q_h - beta q_j by at most one
         // rounding per component
-        nd += 0x1p-20f * (nh + beta * sqrtf(nj2));
+        nd += 0x1p-20f * (nh + beta * nj);
         if (lane == 0) wt[best] += wh * beta;
       }
       C += fabsf(wh) * nd;
       // x_h = w_h d_h (the FP32 residual; the joint bound's slack below covers
-      // its rounding), its Gram terms with the earlier residuals, and the sum
-      float x[4];
+      // its rounding)
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        float d = v[m];
-#pragma unroll
-        for (int j = 0; j < kPruneR; ++j)
-          if (j == best) d = fmaf(-beta, kept[j][m], v[m]);
-        x[m] = m < per ? wh * d : 0.f;
-        xsum[m] += x[m];
+        const float x = m < per ? wh * d[m] : 0.f;
+        xsum[m] += x;
+        gdiag = fmaf(x, x, gdiag);
+        if (m < per) xs[h - kPruneR][lane + 32 * m] = x;
       }
-      float xx = 0.f;
-#pragma unroll
-      for (int m = 0; m < 4; ++m) xx = fmaf(x[m], x[m], xx);
-      G += warp_sum_f32(xx);
-      for (int l = 0; l < h - kPruneR; ++l) {
-        float dd = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-          if (m < per) dd = fmaf(x[m], xs[l][lane + 32 * m], dd);
-        G += 2.f * fabsf(warp_sum_f32(dd));
-      }
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        if (m < per) xs[h - kPruneR][lane + 32 * m] = x[m];
       __syncwarp();
     }
+    // off-diagonal Gram terms: lane l of round h takes the pairs (h, l + 32 i)
+    float goff = 0.f;
+    const int nx = H - kPruneR;
+    for (int h = 1; h < nx; ++h)
+      for (int l = lane; l < h; l += 32) goff += 2.f * fabsf(row_dot(xs[h], xs[l], D));
+    const float G = warp_sum_f32(gdiag) + warp_sum_f32(goff);
     float sx = 0.f;
 #pragma unroll
     for (int m = 0; m < 4; ++m) sx = fmaf(xsum[m], xsum[m], sx);
@@ -183,6 +197,7 @@ __global__ void __launch_bounds__(32) prune_prep_kernel(const void* __restrict__
     const float resid = fminf(round_up_pos(C), joint);
     const float ceff = round_up_pos(resid + 0x1p-11f * wsum);
     float* o = out + static_cast<size_t>(t) * (kPruneR + 2);
+    __syncwarp();
     if (lane < kPruneR) o[lane] = wt[lane];
     if (lane == 0) {
       o[kPruneR] = ceff;

@@ -133,13 +133,21 @@ __global__ void __launch_bounds__(kSeedThreads) witness_scores_kernel(const Witn
         for (int h = 0; h < H; ++h) {
           const float4* qh = reinterpret_cast<const float4*>(qs + h * D);
           float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;  // four independent chains
+          // 32 dims at a time: eight shared-memory loads in flight, then their
+          // 32 multiply-adds
 #pragma unroll
-          for (int d4 = 0; d4 < D / 4; ++d4) {
-            const float4 v = qh[d4];
-            x0 = fmaf(v.x, kr[4 * d4], x0);
-            x1 = fmaf(v.y, kr[4 * d4 + 1], x1);
-            x2 = fmaf(v.z, kr[4 * d4 + 2], x2);
-            x3 = fmaf(v.w, kr[4 * d4 + 3], x3);
+          for (int blk = 0; blk < D / 32; ++blk) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = qh[8 * blk + u];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int d = 32 * blk + 4 * u;
+              x0 = fmaf(v[u].x, kr[d], x0);
+              x1 = fmaf(v[u].y, kr[d + 1], x1);
+              x2 = fmaf(v[u].z, kr[d + 2], x2);
+              x3 = fmaf(v[u].w, kr[d + 3], x3);
+            }
           }
           s = fmaf(ws[h], fmaxf((x0 + x1) + (x2 + x3), 0.f), s);
         }
