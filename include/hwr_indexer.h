@@ -197,8 +197,8 @@ indexer_status indexer_topk_host(const indexer_problem* p, const void* q, const 
  *          indices for COMPRESSED.  The previous decode step's out_idx row is
  *          a typical seed row.  Entries that are negative or not visible to
  *          the query are ignored, and so is any entry naming a key at or below
- *          the largest key named earlier in its row (so rows in ascending
- *          order are used whole, and no key counts twice).
+ *          the largest visible key named earlier in its row (so rows in
+ *          ascending order are used whole, and no key counts twice).
  * Each row's remaining seeds are scored exactly in FP32 on CUDA cores,
  * lowered by a margin that covers the difference to the tensor-core scores
  * (eps |k| sum_h |w_h||q_h| with eps = 2^-12 for BF16 and 2^-9 for FP8, times

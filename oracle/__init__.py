@@ -26,6 +26,8 @@ from .indexer_oracle import (  # noqa: F401
     out_width,
     topk_rows,
     topk_rows_docs,
+    witness_seed_keys,
+    witness_threshold,
     decode_keys_for,
     pair_shared_counts,
     pair_regions,

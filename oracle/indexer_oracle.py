@@ -317,6 +317,60 @@ def topk_rows(problem: dict, q_rows, k, w_rows, rows, q_scale_rows=None,
     return out_idx, out_len, out_score, taus
 
 
+def witness_seed_keys(seed_row, g: int, n_keys: int, visibility: int, ratio: int) -> np.ndarray:
+    """The distinct visible key rows that one row of seeds names, in order.
+
+    [DoSA] 核心方法 (first step) scores a set of at least K visible seed keys
+    exactly; a key counted twice would make its K-th score too high, so each
+    key counts once.  An entry e names key row e (for POOLED a token position,
+    which names the pool e // ratio holding it).  An entry is dropped when it
+    is negative, when the key it names is not visible at g, or when that key is
+    at or below the largest key kept so far (rows in ascending order are used
+    whole).
+    """
+    n_vis = visible_keys(g, n_keys, visibility, ratio).size   # the visible keys are 0 .. n_vis-1
+    kept = []
+    top = -1
+    for e in np.asarray(seed_row).tolist():
+        if e < 0:
+            continue
+        r = e // ratio if visibility == POOLED else e
+        if r >= n_vis or r <= top:
+            continue
+        kept.append(r)
+        top = r
+    return np.asarray(kept, dtype=np.int64)
+
+
+def witness_threshold(problem: dict, q_rows, k, w_rows, rows, seeds, q_scale_rows=None,
+                      k_scale=None, pool_coef=None, keys_f64=None) -> np.ndarray:
+    """tau[r]: the K-th largest exact score over the distinct visible seeds of
+    query row rows[r] ([DoSA] 核心方法, first step: a lower bound of the row's
+    K-th score, since those seeds are some of its visible keys), NaN when the
+    row has fewer than K (K / ratio pools for POOLED) such seeds.
+    Arguments as topk_rows, plus seeds [R, n] (one row of seeds per query row).
+    """
+    vis_mode = problem["visibility"]
+    ratio = int(problem["ratio"]) if vis_mode != TOKEN else 1
+    K = int(problem["K"])
+    ksel = K // ratio if vis_mode == POOLED else K
+    if keys_f64 is None:
+        keys_f64 = _decode_keys(problem, k, k_scale, pool_coef)
+    taus = np.full(len(rows), math.nan, dtype=np.float64)
+    for r in range(len(rows)):
+        g = int(problem["q_pos0"]) + int(rows[r])
+        sk = witness_seed_keys(seeds[r], g, keys_f64.shape[0], vis_mode, ratio)
+        if sk.size < ksel:
+            continue
+        if problem["dtype"] == "fp8":
+            q_t = decode_e4m3(q_rows[r]) * np.asarray(q_scale_rows[r], dtype=np.float64)[:, None]
+        else:
+            q_t = decode_bf16(q_rows[r])
+        s = score_keys(q_t, np.asarray(w_rows[r], dtype=np.float64), keys_f64[sk])
+        taus[r] = float(np.sort(s)[::-1][ksel - 1])
+    return taus
+
+
 def topk_rows_docs(problem: dict, q_rows, k, w_rows, rows, doc_bounds, q_scale_rows=None,
                    k_scale=None, pool_coef=None):
     """Indexer output for query rows of a packed batch of documents.

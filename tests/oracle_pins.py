@@ -503,6 +503,46 @@ def pin_fp8_scales(O):
     assert i1[0, : l1[0]].tolist() == sorted(top.tolist())
 
 
+def pin_witness(O):
+    """Seed threshold ([DoSA] 核心方法, first step): the seed rule by hand
+    (negative, invisible and repeated or out-of-order keys dropped; a pooled
+    position names its pool); seeds equal to the row's own top-K give exactly
+    its K-th score; any K or more distinct visible seeds give at most that
+    (brute force over the full score row); K copies of one key are one seed."""
+    assert O.witness_seed_keys([5, 3, 5, 7, -1, 10**9, 8], 100, 50, O.TOKEN, 1).tolist() == [5, 7, 8]
+    assert O.witness_seed_keys([8, 9, 10, 11, 12, 13, 14], 13, 100, O.POOLED, 4).tolist() == [2]
+    assert O.witness_seed_keys([0, 2, 3, 1], 13, 100, O.COMPRESSED, 4).tolist() == [0, 2]
+    rng = np.random.default_rng(41)
+    H, D, T, K = 3, 8, 60, 6
+    qb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, H, D)))
+    kb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, D)))
+    w = rng.integers(-2, 3, size=(T, H)).astype(np.float32)
+    rows = np.arange(T)
+    prob = _problem(S=T, T=T, H=H, D=D, K=K)
+    idx, ln, _, tau = O.topk_rows(prob, qb, kb, w, rows)
+    got = O.witness_threshold(prob, qb, kb, w, rows, idx)
+    full = ln == K
+    assert np.array_equal(got[full], tau[full]) and np.isnan(got[~full]).all()
+    keys = O.decode_bf16(kb)
+    for t in range(K, T):
+        s = np.sort(O.score_keys(O.decode_bf16(qb[t]), w[t].astype(np.float64), keys[: t + 1]))[::-1]
+        for _ in range(3):
+            n = int(rng.integers(K, t + 2))
+            seeds = np.sort(rng.choice(t + 1, size=n, replace=False))
+            sub = np.sort(O.score_keys(O.decode_bf16(qb[t]), w[t].astype(np.float64), keys[seeds]))[::-1]
+            th = O.witness_threshold(prob, qb[t:t + 1], kb, w[t:t + 1], [t], seeds[None, :])[0]
+            assert th == sub[K - 1] and th <= s[K - 1]
+    best = int(np.argmax(O.score_keys(O.decode_bf16(qb[T - 1]), w[T - 1].astype(np.float64), keys)))
+    assert np.isnan(O.witness_threshold(prob, qb[-1:], kb, w[-1:], [T - 1], np.full((1, K), best))[0])
+    # pooled: the row's own output (token positions, then the tail) gives its K-th pool score
+    c = _bf16_bits_of_ints(rng.integers(0, 3, size=(4, D)))
+    pprob = _problem(S=T, T=T, H=H, D=D, K=8, vis=O.POOLED, ratio=4)
+    pidx, pln, _, ptau = O.topk_rows(pprob, qb, kb, w, rows, pool_coef=c)
+    pgot = O.witness_threshold(pprob, qb, kb, w, rows, pidx, pool_coef=c)
+    pfull = ~np.isnan(ptau)
+    assert pfull.any() and np.array_equal(pgot[pfull], ptau[pfull]) and np.isnan(pgot[~pfull]).all()
+
+
 PINS = [
     pin_hand_worked,
     pin_integer_bruteforce,
@@ -522,4 +562,5 @@ PINS = [
     pin_pair_regions,
     pin_documents,
     pin_fp8_scales,
+    pin_witness,
 ]

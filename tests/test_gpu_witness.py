@@ -152,3 +152,48 @@ def test_witness_rejects_bad_arguments(cuda_ok):
     with pytest.raises(I.IndexerError) as e:
         I.indexer_topk_witness(prob, inp["q"], inp["k"], inp["w"], None, None, None, seeds, idx, ln, None, small)
     assert e.value.status == 2   # INDEXER_EWORKSPACE
+
+
+def test_witness_threshold_against_oracle(cuda_ok):
+    """The threshold the seed kernels compute (kept after the indexer's own
+    workspace and the seed scores) is a lower bound of the oracle's exact K-th
+    score over the row's distinct visible seeds, within twice the rounding
+    margin of it; rows with fewer than K such seeds get no threshold (0)."""
+    import oracle
+    from head_weighted_relu_b200 import indexer as I
+    wl = W.Workload("wit_thr", S=8, T=30000, H=64, D=128, K=512, q_pos0=30000 - 8, seed=102)
+    inp = W.generate(wl, "cuda")
+    ref = _plain(wl, inp)
+    # even rows: their own selection (a tight threshold); odd rows: the row
+    # above's (a loose one); the last row: half a row (too few seeds)
+    seeds = torch.where((torch.arange(wl.S, device="cuda") % 2 == 0)[:, None], ref[0], torch.roll(ref[0], 1, 0))
+    seeds[-1, wl.K // 2:] = -1
+    seeds = seeds.contiguous()
+    prob = _problem(wl)
+    n = seeds.shape[1]
+    ws = torch.empty(I.indexer_witness_workspace_bytes(prob, n), dtype=torch.uint8, device="cuda")
+    idx = torch.empty_like(ref[0])
+    ln = torch.empty_like(ref[1])
+    I.indexer_topk_witness(prob, inp["q"], inp["k"], inp["w"], None, None, None, seeds, idx, ln, None, ws)
+    torch.cuda.synchronize()
+    assert I.indexer_read_status(ws) == 0
+    off = I.indexer_workspace_bytes(prob) + (wl.S * n * 4 + 255) // 256 * 256
+    thr = ws[off: off + 4 * wl.S].cpu().numpy().view(np.uint32)
+    bits = np.where(thr & 0x80000000, thr & 0x7FFFFFFF, ~thr).astype(np.uint32)
+    thr_f = bits.view(np.float32).astype(np.float64)
+
+    rows = np.arange(wl.S, dtype=np.int64)
+    h = parity.host_inputs(inp, rows)
+    s_np = seeds.cpu().numpy()
+    tau = oracle.witness_threshold(wl.problem(), h["q_rows"], h["k"], h["w_rows"], rows, s_np)
+    keys = oracle.decode_keys_for(wl.problem(), h["k"])
+    assert np.isnan(tau[-1]) and thr[-1] == 0
+    for t in range(wl.S - 1):
+        assert not np.isnan(tau[t])
+        q_t = oracle.decode_bf16(h["q_rows"][t])
+        amp = float(np.abs(h["w_rows"][t].astype(np.float64)) @ np.linalg.norm(q_t, axis=1))
+        sk = oracle.witness_seed_keys(s_np[t], wl.q_pos0 + t, keys.shape[0], W.TOKEN, 1)
+        kmax = float(np.linalg.norm(keys[sk], axis=1).max())
+        margin = 2.0 ** -12 * kmax * amp
+        assert thr_f[t] <= tau[t], (t, thr_f[t], tau[t])
+        assert thr_f[t] >= tau[t] - 2 * margin - 1e-5 * abs(tau[t]), (t, thr_f[t], tau[t], margin)

@@ -38,6 +38,9 @@ MUTATIONS = {
     "pools_from_global_grid": ("            pos = (b + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)",
                                "            pos = (b // ratio * ratio + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)"),
     "regions_unsorted": ("            ordered = sorted(members)", "            ordered = sorted(members, reverse=True)"),
+    "witness_counts_repeats": ("        if r >= n_vis or r <= top:", "        if r >= n_vis:"),
+    "witness_counts_invisible": ("        if r >= n_vis or r <= top:", "        if r <= top:"),
+    "witness_kth_off_by_one": ("taus[r] = float(np.sort(s)[::-1][ksel - 1])", "taus[r] = float(np.sort(s)[::-1][ksel - 2])"),
 }
 
 
