@@ -541,6 +541,23 @@ def pin_witness(O):
     pgot = O.witness_threshold(pprob, qb, kb, w, rows, pidx, pool_coef=c)
     pfull = ~np.isnan(ptau)
     assert pfull.any() and np.array_equal(pgot[pfull], ptau[pfull]) and np.isnan(pgot[~pfull]).all()
+    # compressed keys and FP8 storage: the row's own output again gives its K-th score
+    cprob = _problem(S=T, T=T // 4, H=H, D=D, K=4, vis=O.COMPRESSED, ratio=4)
+    cidx, _, _, ctau = O.topk_rows(cprob, qb, kb[: T // 4], w, rows)
+    cgot = O.witness_threshold(cprob, qb, kb[: T // 4], w, rows, cidx)
+    cfull = ~np.isnan(ctau)
+    assert cfull.any() and np.array_equal(cgot[cfull], ctau[cfull]) and np.isnan(cgot[~cfull]).all()
+    codes_q = rng.integers(0, 0x7E, size=(4, H, D)).astype(np.uint8)
+    codes_k = rng.integers(0, 0x7E, size=(T, D)).astype(np.uint8)
+    codes_k[::2] |= 0x80
+    qs = rng.uniform(0.5, 2.0, size=(4, H)).astype(np.float32)
+    ks = rng.uniform(0.5, 2.0, size=T).astype(np.float32)
+    fprob = _problem(S=4, T=T, H=H, D=D, K=K, dtype="fp8", q_pos0=T - 4)
+    fidx, _, _, ftau = O.topk_rows(fprob, codes_q, codes_k, w[:4], np.arange(4), q_scale_rows=qs, k_scale=ks)
+    fgot = O.witness_threshold(fprob, codes_q, codes_k, w[:4], np.arange(4), fidx, q_scale_rows=qs, k_scale=ks)
+    # non-integer values: the two paths score different key subsets, so allow
+    # a difference in the last bits of the FP64 sums
+    assert np.allclose(fgot, ftau, rtol=1e-12, atol=0.0) and not np.isnan(fgot).any()
 
 
 PINS = [
