@@ -305,23 +305,121 @@ def pin_pooled_keys(O):
             assert int(kp[p, d]) == _nearest_bf16_bits(exact), (p, d)
 
 
+def pooled_rounding_cases():
+    """Columns of tests/golden/pooled_rounding_cases.txt: (k [4] values,
+    c [4] values, expected bfloat16 bits), values as exact Fractions."""
+    out = []
+    with open(os.path.join(GOLDEN, "pooled_rounding_cases.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            nums = [int(x) for x in parts[:16]]
+            vals = [Fraction(nums[2 * i]) * Fraction(2) ** nums[2 * i + 1] for i in range(8)]
+            out.append((vals[:4], vals[4:], int(parts[16], 0)))
+    return out
+
+
+def _bf16_bits_of_fractions(vals) -> np.ndarray:
+    """Exact bfloat16 values (as Fractions) -> bit patterns, through torch."""
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64).to(torch.bfloat16)
+    back = t.double().numpy()
+    assert all(Fraction(float(b)) == v for b, v in zip(back, vals)), "not a bfloat16 value"
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def wide_pool_columns(n_cols: int, seed: int):
+    """Random pool columns (k [n_cols pools of 4 tokens, 1 channel] and c
+    [4, n_cols]) whose products span up to 2^80 in magnitude, so that most
+    binary64 running sums are inexact.  Returns bf16 bits k [4 * n, 1] laid
+    out as n pools of one channel, and c [4, 1] per column as a list."""
+    rng = np.random.default_rng(seed)
+    mant = rng.integers(1, 256, size=(n_cols, 8)) * rng.choice([-1, 1], size=(n_cols, 8))
+    expo = rng.integers(-40, 41, size=(n_cols, 8))
+    return [[Fraction(int(m)) * Fraction(2) ** int(e) for m, e in zip(mant[i], expo[i])] for i in range(n_cols)]
+
+
+def pin_pooled_keys_inexact_sums(O):
+    """Pool keys whose binary64 running sum is inexact ("Module 06 — DSA &
+    KPool", §2; one RNE rounding of the exact sum): the hand-worked columns of
+    tests/golden/pooled_rounding_cases.txt (ties hidden by cancelling terms,
+    subnormal and overflowing results, a cancellation a double-double
+    accumulation gets wrong) and random columns with exponent spreads up to
+    2^80, each against the nearest bfloat16 of the exact rational sum."""
+    cases = pooled_rounding_cases()
+    # one column per case: c varies by channel, so each case gets its own channel
+    D = len(cases)
+    k = np.zeros((4, D), dtype=np.uint16)
+    c = np.zeros((4, D), dtype=np.uint16)
+    for d, (kv, cv, _) in enumerate(cases):
+        k[:, d] = _bf16_bits_of_fractions(kv)
+        c[:, d] = _bf16_bits_of_fractions(cv)
+    got = O.pooled_keys(k, c, 4)
+    assert got.shape == (1, D)
+    for d, (kv, cv, want) in enumerate(cases):
+        exact = sum(a * b for a, b in zip(kv, cv))
+        assert _nearest_bf16_bits(exact) == want, (d, hex(want))
+        assert int(got[0, d]) == want, (d, hex(int(got[0, d])), hex(want))
+    # random wide columns: every pool of a channel shares that channel's c
+    cols = wide_pool_columns(240, seed=19)
+    n_pools, D = 6, len(cols) // 6
+    k = np.zeros((4 * n_pools, D), dtype=np.uint16)
+    c = np.zeros((4, D), dtype=np.uint16)
+    inexact = 0
+    for d in range(D):
+        c[:, d] = _bf16_bits_of_fractions(cols[d * n_pools][4:])
+        for p in range(n_pools):
+            k[4 * p: 4 * p + 4, d] = _bf16_bits_of_fractions(cols[d * n_pools + p][:4])
+    got = O.pooled_keys(k, c, 4)
+    kf = [[Fraction(float(x)) for x in row] for row in O.decode_bf16(k).tolist()]
+    cf = [[Fraction(float(x)) for x in row] for row in O.decode_bf16(c).tolist()]
+    for p in range(n_pools):
+        for d in range(D):
+            exact = sum(kf[4 * p + j][d] * cf[j][d] for j in range(4))
+            fsum = 0.0
+            for j in range(4):
+                fsum += float(kf[4 * p + j][d] * cf[j][d])
+            inexact += Fraction(fsum) != exact
+            assert int(got[p, d]) == _nearest_bf16_bits(exact), (p, d)
+    assert inexact >= 60, inexact   # most columns exercise the exact-sum fallback
+
+
+_LADDER = []
+
+
+def _bf16_ladder():
+    """Every non-negative finite bfloat16 value as a Fraction, in pattern order,
+    then 2^128 for the infinity pattern (built once)."""
+    if not _LADDER:
+        vals = torch.arange(0, 0x7F80, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).double().numpy()
+        _LADDER.extend(Fraction(float(x)) for x in vals)
+        _LADDER.append(Fraction(2) ** 128)
+    return _LADDER
+
+
 def _nearest_bf16_bits(v: Fraction) -> int:
     """Nearest bfloat16 to an exact rational (ties to the even pattern), found
-    by bisection over the ordered positive bit patterns, decoded by torch."""
+    by bisection over the ordered positive bit patterns, decoded by torch.
+    The infinity pattern 0x7F80 stands for 2^128 (IEEE overflow under
+    round-to-nearest: at or above the largest finite value plus half its
+    spacing the result is infinite)."""
     if v == 0:
         return 0
     sign = 0x8000 if v < 0 else 0
     a = abs(v)
-    pats = torch.arange(0, 0x7F80, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float().numpy()
+    pats = _bf16_ladder()
+    if a >= pats[-1]:
+        return sign | 0x7F80
     lo, hi = 0, len(pats) - 1
     while hi - lo > 1:
         mid = (lo + hi) // 2
-        if Fraction(float(pats[mid])) <= a:
+        if pats[mid] <= a:
             lo = mid
         else:
             hi = mid
-    dl = a - Fraction(float(pats[lo]))
-    dh = Fraction(float(pats[hi])) - a
+    dl = a - pats[lo]
+    dh = pats[hi] - a
     if dl < dh or (dl == dh and lo % 2 == 0):
         return sign | lo
     return sign | hi
@@ -474,6 +572,43 @@ def pin_documents(O):
                                           for i in range(0, len(body), 4)), t
 
 
+def pin_documents_compressed(O):
+    """Compressed keys in a packed batch ("Module 06 — DSA & KPool", §3 and
+    "Ship it": nothing of one document may reach another's selection): a
+    document starts on a whole compressed key, and the query at global
+    position g in the document starting at token b sees compressed key j iff
+    j >= b / ratio and ratio*j + ratio - 1 <= g.  Checked by brute force: the
+    full score row over every compressed key, every other key excluded, a
+    stable sort; a batch of one document equals the plain compressed indexer;
+    a query within ratio - 1 tokens of its document start selects nothing."""
+    rng = np.random.default_rng(43)
+    H, D, m, K = 3, 8, 4, 5
+    n_tok = 64
+    T = n_tok // m
+    qb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(n_tok, H, D)))
+    kb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(T, D)))
+    w = rng.integers(-2, 3, size=(n_tok, H)).astype(np.float32)
+    rows = np.arange(n_tok)
+    prob = _problem(S=n_tok, T=T, H=H, D=D, K=K, vis=O.COMPRESSED, ratio=m)
+    a = O.topk_rows(prob, qb, kb, w, rows)
+    b = O.topk_rows_docs(prob, qb, kb, w, rows, [0, n_tok])
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    bounds = [0, 12, 16, 40, 64]   # documents of 12, 4, 24 and 24 tokens
+    idx, ln, _, _ = O.topk_rows_docs(prob, qb, kb, w, rows, bounds)
+    keys = O.decode_bf16(kb)
+    for t in rows:
+        d = int(np.searchsorted(bounds, t, side="right")) - 1
+        start = bounds[d]
+        s = O.score_keys(O.decode_bf16(qb[t]), w[t].astype(np.float64), keys)
+        allowed = np.array([j * m >= start and m * j + m - 1 <= t for j in range(T)])
+        s[~allowed] = -np.inf
+        n = min(K, int(allowed.sum()))
+        top = np.argsort(-s, kind="stable")[:n]
+        assert idx[t, : ln[t]].tolist() == sorted(top.tolist()), t
+        if t - start < m - 1:
+            assert ln[t] == 0, t
+
+
 def pin_fp8_scales(O):
     """An FP8 value means code * row scale: doubling every key scale doubles
     every score and leaves the selection unchanged; a per-(query, head) scale
@@ -573,11 +708,13 @@ PINS = [
     pin_watch_lengths,
     pin_slot_count,
     pin_pooled_keys,
+    pin_pooled_keys_inexact_sums,
     pin_e4m3_decoder,
     pin_bf16_codec,
     pin_pair_overlap,
     pin_pair_regions,
     pin_documents,
+    pin_documents_compressed,
     pin_fp8_scales,
     pin_witness,
 ]

@@ -40,6 +40,14 @@ MUTATIONS = {
     "regions_unsorted": ("            ordered = sorted(members)", "            ordered = sorted(members, reverse=True)"),
     "witness_counts_repeats": ("        if r >= n_vis or r <= top:", "        if r >= n_vis:"),
     "witness_counts_invisible": ("        if r >= n_vis or r <= top:", "        if r <= top:"),
+    "fraction_ties_to_odd": ("rem == Fraction(1, 2) and n % 2 == 1", "rem == Fraction(1, 2) and n % 2 == 0"),
+    "fraction_fallback_dropped": ("        out[p, dd] = _round_fraction_to_bf16_bits(exact)",
+                                  "        out[p, dd] = out[p, dd]"),
+    "fraction_subnormal_spacing": ("quantum = Fraction(2) ** (max(e, -126) - 7)", "quantum = Fraction(2) ** (e - 7)"),
+    "compressed_doc_start_exclusive": ("vis = j[(j >= b // ratio) & (ratio * j + ratio - 1 <= g)]",
+                                       "vis = j[(j > b // ratio) & (ratio * j + ratio - 1 <= g)]"),
+    "compressed_doc_start_ignored": ("vis = j[(j >= b // ratio) & (ratio * j + ratio - 1 <= g)]",
+                                     "vis = j[(ratio * j + ratio - 1 <= g)]"),
     "witness_kth_off_by_one": ("taus[r] = float(np.sort(s)[::-1][ksel - 1])", "taus[r] = float(np.sort(s)[::-1][ksel - 2])"),
 }
 
