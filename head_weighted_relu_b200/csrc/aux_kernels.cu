@@ -26,27 +26,99 @@ __device__ __forceinline__ uint16_t cvt_rn_bf16_f64(double x) {
   return r;
 }
 
-// Round hi + lo (|lo| at most half an ulp of hi, the pair an error-free sum)
-// to bfloat16, nearest-even.  Rounding hi alone is right unless hi sits exactly
-// halfway between two bfloat16 values; then the sign of lo decides.
-__device__ __forceinline__ uint16_t round_pair_to_bf16(double hi, double lo) {
-  if (lo != 0.0 && hi != 0.0) {
-    int e;
-    frexp(hi, &e);                          // |hi| = f * 2^e, 0.5 <= f < 1
-    const int qexp = max(e - 8, -133);      // bfloat16 spacing at |hi|: 2^qexp
-    const double halves = ldexp(hi, 1 - qexp);  // hi in units of half a spacing (exact)
-    const double r = rint(halves);
-    if (r == halves && fmod(fabs(r), 2.0) == 1.0) {  // exactly halfway
-      const double half = ldexp(1.0, qexp - 1);
-      return cvt_rn_bf16_f64(lo > 0.0 ? hi + half : hi - half);
-    }
-  }
-  return cvt_rn_bf16_f64(hi);
+// Exact summation and rounding of pool keys.  Each product of two bfloat16
+// values is exact in binary64, so the sum of a pool's products is an exact
+// rational that a binary64 running sum may round (for example 2^60 + 1 - 2^60
+// - 1 or 259*2^52 - 2^-60).  When every addition is exact the running sum is
+// rounded directly; otherwise the sum is kept as a nonoverlapping expansion
+// (Shewchuk, "Adaptive Precision Floating-Point Arithmetic and Fast Robust
+// Geometric Predicates", 1997: TwoSum and Grow-Expansion), whose sign is the
+// sign of its largest nonzero component, and the bfloat16 rounding is decided
+// by exact comparisons with the midpoints next to a near candidate.
+
+constexpr int kMaxPoolRatio = 16;
+constexpr int kExpMax = kMaxPoolRatio + 1;   // products, plus one midpoint
+
+__device__ __forceinline__ void two_sum(double a, double b, double& s, double& err) {
+  s = __dadd_rn(a, b);
+  const double bb = __dsub_rn(s, a);
+  err = __dadd_rn(__dsub_rn(a, __dsub_rn(s, bb)), __dsub_rn(b, bb));
 }
 
-// kp[p, d] = RNE_bf16( sum_j c[j, d] * k[ratio*p + j, d] ), the sum exact:
-// each product of two bfloat16 values is exact in binary64 and the running
-// sum is kept as an unevaluated pair (hi, lo) with Knuth's TwoSum.
+// e[0, n) nonoverlapping, increasing magnitude (zeros allowed) -> the same
+// for e + b, one component longer.
+__device__ __forceinline__ void grow_expansion(double (&e)[kExpMax], int& n, double b) {
+  double q = b;
+#pragma unroll
+  for (int i = 0; i < kExpMax; ++i) {
+    if (i < n) {
+      double h;
+      two_sum(q, e[i], q, h);
+      e[i] = h;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kExpMax; ++i)
+    if (i == n) e[i] = q;
+  ++n;
+}
+
+// Sign (-1, 0, 1) of the exact value of a nonoverlapping expansion: the sign
+// of its largest nonzero component, which is the last one.
+__device__ __forceinline__ int expansion_sign(const double (&e)[kExpMax], int n) {
+  int sg = 0;
+#pragma unroll
+  for (int i = 0; i < kExpMax; ++i)
+    if (i < n && e[i] != 0.0) sg = e[i] > 0.0 ? 1 : -1;
+  return sg;
+}
+
+// Sign of (value of e[0, n)) - m, exactly.
+__device__ __forceinline__ int compare_expansion(const double (&e)[kExpMax], int n, double m) {
+  double f[kExpMax];
+#pragma unroll
+  for (int i = 0; i < kExpMax; ++i) f[i] = e[i];
+  int nf = n;
+  grow_expansion(f, nf, -m);
+  return expansion_sign(f, nf);
+}
+
+// Value of a non-negative bfloat16 pattern; the infinity pattern 0x7F80
+// stands for 2^128, where round-to-nearest overflows.
+__device__ __forceinline__ double bf16_pattern_value(uint32_t pat) {
+  return pat >= 0x7F80u ? 0x1p128 : bf16_bits_to_double(static_cast<uint16_t>(pat));
+}
+
+// Round the exact value of e[0, n) (nonzero) to bfloat16, nearest-even.
+__device__ uint16_t round_expansion_to_bf16(double (&e)[kExpMax], int n) {
+  const int sg = expansion_sign(e, n);
+  double approx = 0.0;  // within a few binary64 ulps of the magnitude
+#pragma unroll
+  for (int i = 0; i < kExpMax; ++i) {
+    if (i < n) {
+      if (sg < 0) e[i] = -e[i];
+      approx = __dadd_rn(approx, e[i]);
+    }
+  }
+  // the candidate is the exact answer or one of its neighbours
+  uint32_t pat = cvt_rn_bf16_f64(approx) & 0x7FFFu;
+  if (pat > 0x7F80u) pat = 0x7F80u;
+  const double v = bf16_pattern_value(pat);
+  if (pat < 0x7F80u) {
+    const double up_mid = 0.5 * (v + bf16_pattern_value(pat + 1));
+    const int c = compare_expansion(e, n, up_mid);
+    if (c > 0 || (c == 0 && (pat & 1u))) return static_cast<uint16_t>((sg < 0 ? 0x8000u : 0u) | (pat + 1));
+  }
+  if (pat > 0) {
+    const double lo_mid = 0.5 * (bf16_pattern_value(pat - 1) + v);
+    const int c = compare_expansion(e, n, lo_mid);
+    if (c < 0 || (c == 0 && (pat & 1u))) return static_cast<uint16_t>((sg < 0 ? 0x8000u : 0u) | (pat - 1));
+  }
+  return static_cast<uint16_t>((sg < 0 ? 0x8000u : 0u) | pat);
+}
+
+// kp[p, d] = RNE_bf16( sum_j c[j, d] * k[ratio*p + j, d] ), the sum exact.
+// Inputs are finite; ratio <= kMaxPoolRatio.
 __global__ void pool_keys_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ coef, int ratio,
                                  int64_t n_pools, int D, uint16_t* __restrict__ out) {
   const int64_t n = n_pools * D;
@@ -54,20 +126,27 @@ __global__ void pool_keys_kernel(const uint16_t* __restrict__ k, const uint16_t*
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t pool = e / D;
     const int d = static_cast<int>(e - pool * D);
-    double hi = 0.0, lo = 0.0;
+    double sum = 0.0;
+    bool exact = true;
     for (int j = 0; j < ratio; ++j) {
       const double prod = bf16_bits_to_double(coef[j * D + d]) * bf16_bits_to_double(k[(pool * ratio + j) * D + d]);
-      const double s = __dadd_rn(hi, prod);
-      const double bb = __dsub_rn(s, hi);
-      const double err = __dadd_rn(__dsub_rn(hi, __dsub_rn(s, bb)), __dsub_rn(prod, bb));
-      hi = s;
-      lo = __dadd_rn(lo, err);
+      if (j == 0) {
+        sum = prod;
+      } else {
+        double err;
+        two_sum(sum, prod, sum, err);
+        exact = exact && err == 0.0;
+      }
     }
-    // fold lo into hi once more so that |lo| is below half an ulp of hi
-    const double s = __dadd_rn(hi, lo);
-    const double bb = __dsub_rn(s, hi);
-    const double err = __dadd_rn(__dsub_rn(hi, __dsub_rn(s, bb)), __dsub_rn(lo, bb));
-    out[e] = round_pair_to_bf16(s, err);
+    if (exact) {
+      out[e] = cvt_rn_bf16_f64(sum);  // the running sum is the exact sum (signed zero included)
+      continue;
+    }
+    double ex[kExpMax] = {};
+    int m = 0;
+    for (int j = 0; j < ratio; ++j)
+      grow_expansion(ex, m, bf16_bits_to_double(coef[j * D + d]) * bf16_bits_to_double(k[(pool * ratio + j) * D + d]));
+    out[e] = expansion_sign(ex, m) == 0 ? static_cast<uint16_t>(0) : round_expansion_to_bf16(ex, m);
   }
 }
 

@@ -82,7 +82,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
   if (!p) return INDEXER_EINVAL;
-  if (p->S < 0 || p->T < 1 || p->q_pos0 < 0 || p->K < 1 || (p->flags & ~INDEXER_FLAG_PRUNE) != 0 ||
+  if (p->S < 0 || p->T < 1 || p->q_pos0 < 0 || p->K < 1 ||
+      (p->flags & ~(INDEXER_FLAG_PRUNE | INDEXER_FLAG_TEST_WAIT_TIMEOUT)) != 0 ||
       p->reserved != 0)
     return INDEXER_EINVAL;
   if (p->visibility < INDEXER_VIS_TOKEN || p->visibility > INDEXER_VIS_POOLED) return INDEXER_EINVAL;
@@ -314,6 +315,7 @@ indexer_status run_topk(const indexer_problem* p, const void* q, const void* k, 
   sp.split_kth = split_kth;
   sp.split_rth = split_rth;
   sp.seed_thr = nullptr;
+  sp.test_wait_ns = (p->flags & INDEXER_FLAG_TEST_WAIT_TIMEOUT) ? 1000000 : 0;
   if (seeds) {
     WitnessParams wp;
     wp.S = p->S;

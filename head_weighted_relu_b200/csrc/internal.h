@@ -47,6 +47,7 @@ struct ScoreParams {
   uint32_t* split_rth;   // splits > 1: [S][splits] ordered score of each split's r-th entry, r = ceil(K / splits)
                          // (0 when it has fewer than r)
   const uint32_t* seed_thr;  // [S] ordered-score threshold every query starts from, or null (0 for all)
+  int64_t test_wait_ns;  // > 0: test hook, the MMA issuer waits this long on a barrier nothing arrives at
 };
 
 // Per-variant launch facts, filled by the kernel's translation unit.

@@ -218,6 +218,9 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
   const int etid = threadIdx.x;
   const int lane = etid & 31;
   constexpr int bar_id = 1;
+  // after a wait timeout in the scoring kernel the per-range lists are not
+  // valid (the result is reported invalid through the status word): read none
+  if (*reinterpret_cast<volatile const uint32_t*>(mp.check.status) & kStatusWaitTimeout) return;
   for (int64_t t = blockIdx.x; t < mp.S; t += gridDim.x) {
     const int32_t* cnt = mp.split_cnt + t * mp.splits;
     const uint32_t* kth = mp.split_kth + t * mp.splits;
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int sp = 4 * etid + u;
-      c4[u] = sp < mp.splits ? cnt[sp] : 0;
+      c4[u] = sp < mp.splits ? min(max(cnt[sp], 0), mp.ksel) : 0;
       local += c4[u];
     }
     int32_t incl = local;

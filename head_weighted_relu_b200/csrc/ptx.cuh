@@ -55,8 +55,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up (returns
-// false) after `limit_ns` of wall time or as soon as *abort becomes non-zero,
-// so that a broken pipeline ends the kernel instead of hanging the GPU.
+// false) after `limit_ns` of wall time or, when `abort` is not null, as soon
+// as *abort becomes non-zero, so that a broken pipeline ends the kernel
+// instead of hanging the GPU.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -65,7 +66,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
+    if (abort != nullptr && *abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }

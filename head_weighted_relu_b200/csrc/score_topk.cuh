@@ -80,8 +80,10 @@ struct Barriers {
   uint64_t qfull, qempty;
   uint64_t accfull[2], accempty[2];
   uint64_t mma_done;
+  uint64_t never;      // test hook: a barrier nothing arrives at
   uint32_t tmem_slot;
   int abort;
+  int tmem_busy;       // MMAs may still write TMEM: leave it allocated
 };
 
 template <int H, int D, bool FP8>
@@ -645,7 +647,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->accempty[a], 16);  // one arrival per epilogue warp
     }
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->never, 1);
     bars->abort = 0;
+    bars->tmem_busy = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -663,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kExitBar = 15;
   if (warp < 4) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+  uint32_t n_kloads_done = 0, n_qloads_done = 0;  // loads the producer issued
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -671,6 +676,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t kph = 0, qe_ph = 0;
       bool first = true, ok = true;
+      // loads issued so far: key tiles (stage of each follows from the count)
+      // and q blocks; after an abort the last ones may still be landing
+      uint32_t n_kloads = 0, n_qloads = 0;
       for (int r = 0; ok; ++r) {
         const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
         const int b = it.b;
@@ -682,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
         }
         first = false;
+        ++n_qloads;
         mbar_arrive_expect_tx(&bars->qfull, C::Q_BYTES);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
@@ -689,6 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = it.j0; j < it.j1; ++j) {
           ok = mbar_wait(&bars->kempty[stage], kph ^ 1u, abort_flag, kWaitLimitNs);
           if (!ok) break;
+          ++n_kloads;
           mbar_arrive_expect_tx(&bars->kfull[stage], C::K_STAGE_BYTES);
 #pragma unroll
           for (int bx = 0; bx < C::NBOX; ++bx)
@@ -704,6 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(p.status, kStatusWaitTimeout);
         bars->abort = 1;
       }
+      n_kloads_done = n_kloads;
+      n_qloads_done = n_qloads;
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issuer
@@ -744,11 +756,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(&bars->accfull[a]);
           tc_commit(&bars->kempty[stage]);
+          if (p.test_wait_ns > 0 && tcount == 0) {
+            // test hook: a wait that runs out with an MMA in flight, so that
+            // the whole timeout path below runs
+            ok = mbar_wait(&bars->never, 0u, abort_flag, static_cast<uint64_t>(p.test_wait_ns));
+          }
           ++tcount;
           if (++stage == STAGES) {
             stage = 0;
             kph ^= 1u;
           }
+          if (!ok) break;
         }
         if (!ok) break;
         tc_commit(&bars->qempty);
@@ -757,16 +775,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicOr(p.status, kStatusWaitTimeout);
         bars->abort = 1;
       }
-      // all MMAs issued by this thread have completed before TMEM is freed
+      // every MMA issued by this thread has completed before TMEM is freed:
+      // this wait ignores the abort flag (an MMA in flight always completes)
+      // and only a time limit ends it; if that ever runs out, TMEM stays
+      // allocated rather than being freed under a running MMA
       tc_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0u, abort_flag, kWaitLimitNs);
+      if (!mbar_wait(&bars->mma_done, 0u, nullptr, kWaitLimitNs)) {
+        atomicOr(p.status, kStatusWaitTimeout);
+        bars->tmem_busy = 1;
+      }
     }
   }
   __syncwarp();  // lane 0 of warps 0 and 1 rejoins its warp before the aligned barrier
   tc_fence_before();
   named_bar(kExitBar, kThreads);
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  if (warp == 1 && !*reinterpret_cast<volatile int*>(&bars->tmem_busy)) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // After an abort the consumers may have left loads unconsumed: wait (time
+    // limit only) until every load that can still be in flight has landed, so
+    // that none writes into shared memory after the CTA has exited.  Key load
+    // L went to stage L % STAGES in phase L / STAGES; only the last STAGES can
+    // be pending, and no later phase of their stages was started.
+    const uint32_t first_pending = n_kloads_done > STAGES ? n_kloads_done - STAGES : 0u;
+    for (uint32_t L = first_pending; L < n_kloads_done; ++L)
+      mbar_wait(&bars->kfull[L % STAGES], (L / STAGES) & 1u, nullptr, kWaitLimitNs);
+    if (n_qloads_done > 0) mbar_wait(&bars->qfull, (n_qloads_done - 1) & 1u, nullptr, kWaitLimitNs);
+  }
   } else {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpilogue));
   {

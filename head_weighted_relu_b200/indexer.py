@@ -23,6 +23,7 @@ LIB_PATH = os.environ.get("HWR_INDEXER_LIB") or os.path.join(_HERE, "libhwr_inde
 TOKEN, COMPRESSED, POOLED = 0, 1, 2
 BF16, FP8_E4M3 = 0, 1
 FLAG_PRUNE = 1
+FLAG_TEST_WAIT_TIMEOUT = 1 << 30   # test hook: the kernel's wait-timeout path (outputs not valid)
 
 STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
                 3: "INDEXER_EUNSUPPORTED", 4: "INDEXER_ECUDA", 5: "INDEXER_EDEVICE"}
@@ -104,11 +105,11 @@ def _check(fn, status):
 
 
 def make_problem(S, T, H, D, K, visibility=TOKEN, ratio=1, dtype=BF16, q_pos0=0,
-                 prune=False) -> Problem:
+                 prune=False, flags=0) -> Problem:
     if isinstance(dtype, str):
         dtype = {"bf16": BF16, "fp8": FP8_E4M3}[dtype]
     return Problem(S=S, T=T, H=H, D=D, q_pos0=q_pos0, visibility=visibility, ratio=ratio,
-                   K=K, dtype=dtype, flags=FLAG_PRUNE if prune else 0, reserved=0)
+                   K=K, dtype=dtype, flags=(FLAG_PRUNE if prune else 0) | flags, reserved=0)
 
 
 def indexer_out_width(problem: Problem) -> int:

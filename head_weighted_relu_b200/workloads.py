@@ -19,6 +19,9 @@ Workloads (names carry their sizes):
   long_1m_fp8       T=1,048,576 keys, the last 16,384 positions as queries,
                     H=64, D=128, K=2,048, FP8 e4m3 q and k with per-row FP32
                     scales (amax / 448).
+  pooled_tail_64k   the pooled workload at S=T=65,536 (a profiling-sized case).
+  long_1m_fp8_s2k   the FP8 workload with only the last 2,048 positions as
+                    queries (a profiling-sized case).
   decode_1m_s16     16 query rows at the end of T=1,048,576 keys (a decode step
                     of 16 sequences' worth of indexer queries against one long
                     context), H=64, D=128, K=2,048, bf16: the split key-range
@@ -76,6 +79,12 @@ WORKLOADS = {
     "long_1m_fp8": Workload("long_1m_fp8", S=16384, T=1048576, H=64, D=128,
                             K=2048, dtype="fp8", q_pos0=1048576 - 16384,
                             seed=4, pair_overlap=True),
+    "pooled_tail_64k": Workload("pooled_tail_64k", S=65536, T=65536, H=32,
+                                D=128, K=2048, visibility=POOLED, ratio=4,
+                                seed=7),
+    "long_1m_fp8_s2k": Workload("long_1m_fp8_s2k", S=2048, T=1048576, H=64,
+                                D=128, K=2048, dtype="fp8",
+                                q_pos0=1048576 - 2048, seed=8),
     "decode_1m_s16": Workload("decode_1m_s16", S=16, T=1048576, H=64, D=128,
                               K=2048, q_pos0=1048576 - 16, seed=6),
 }

@@ -80,7 +80,7 @@ typedef struct {
   int32_t ratio;      /* m for COMPRESSED / POOLED (1..16); ignored for TOKEN */
   int32_t K;          /* budget in positions; POOLED selects K/ratio pools    */
   int32_t dtype;      /* indexer_dtype                                        */
-  int32_t flags;      /* 0, or INDEXER_FLAG_PRUNE                             */
+  int32_t flags;      /* 0, INDEXER_FLAG_PRUNE (and the test hook below)     */
   int32_t reserved;   /* must be 0                                            */
 } indexer_problem;
 
@@ -97,6 +97,17 @@ typedef struct {
  * bit-identical to the run without the flag.  Needs H >= 32, D % 32 == 0,
  * D <= 128; adds two small set-up kernels and workspace. */
 enum { INDEXER_FLAG_PRUNE = 1 };
+
+/* Test hook for the kernel's failure path (not for production use).  With
+ * this flag every CTA of the scoring kernel, right after issuing its first
+ * tile's MMAs, waits on a barrier that nothing ever arrives at, for about one
+ * millisecond.  The wait runs out, the kernel takes the same exit as after any
+ * pipeline wait that gives up -- the other roles see the abort, in-flight
+ * MMAs and tensor loads are awaited before TMEM is freed and the CTA exits --
+ * and bit 0 of the status word is set (indexer_read_status).  The outputs are
+ * not valid; the device stays usable for the next call.  (Bounded device waits
+ * with an error status: no device fault, trap or endless loop is used.) */
+enum { INDEXER_FLAG_TEST_WAIT_TIMEOUT = 1 << 30 };
 
 /* Row width of out_idx / out_score: K, or K + ratio - 1 for POOLED (2,051 for
  * K = 2,048 and pools of 4; KPool §2, "size index buffers to 2,051").
