@@ -1,18 +1,30 @@
 """Benchmark of the indexer hot path (score + top-K + finalise) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--scaling strong|weak] [--impl ours|reference]
 
-One step = one indexer_topk call over the whole workload (every query row),
-inputs resident in HBM.  Prints one JSON line (rank 0).  Under torchrun each
-rank runs its own independent problem of the same shape (weak scaling); the
-time is the max over ranks.
+One step = one indexer_topk call over the whole workload (every query row; the
+FP8 long-context workload adds the pair-overlap count), inputs resident in
+HBM.  Prints one JSON line (rank 0).
+
+Under torchrun (N > 1) the default is strong scaling: the workload's query
+rows are split across the ranks by visible-pair count (indexer_partition_rows),
+keys replicated on every GPU (each rank draws the same seeded inputs), and
+each rank runs the indexer on its rows; nothing is exchanged.  `value` is the
+whole problem's pairs / the max over ranks of the device time.  --scaling weak
+gives every rank its own problem of the workload's shape instead.
+
+At N = 1 the line also carries `configs`: the same measurement (fewer steps)
+for every configuration the indexer is quoted on, and `cpu_baseline`: the FP64
+oracle on the host's cores over the 1,024 seeded query rows the parity tests
+check (all cores, and one core), with an extrapolated full-problem time.
 """
 
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -25,10 +37,12 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from head_weighted_relu_b200 import workloads as W  # noqa: E402
+from head_weighted_relu_b200 import workloads as W  # noqa: E402  (no library load)
 
 METRIC = "indexer Gpairs/s (causal q·k pairs scored+top-K'd) & % tensor peak; peak HBM GB"
-L2_BYTES = 126 * 2 ** 20
+# the configurations the indexer's metric is quoted on (tiny exactness case,
+# token prefill, compressed keys, pooled keys with tail, 1M-key FP8 chunk)
+QUOTED_CONFIGS = ("tiny_int_512", "dsa_prefill_64k", "csa_m4_256k", "pooled_tail_128k", "long_1m_fp8")
 
 
 def _peaks():
@@ -47,6 +61,7 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.lines = []
 
     def __enter__(self):
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -69,7 +84,6 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -81,7 +95,7 @@ class ClockSampler:
     def summary(self):
         mhz, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -122,179 +136,288 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def rank_workload(wl, rank):
-    """Each rank's independent problem: the workload's shape, its own seed."""
-    return wl.scaled(seed=wl.seed + 1000 * rank)
+# ---------------------------------------------------------------------------
+# Work accounting and the split of one problem across ranks
+# ---------------------------------------------------------------------------
+
+def visible_per_row(wl, rows=None) -> np.ndarray:
+    """Keys (pools for pooled keys) visible to each query row: the pairs the
+    indexer scores for that row."""
+    t = np.arange(wl.S, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    g = t + wl.q_pos0
+    if wl.visibility == W.TOKEN:
+        return np.minimum(g + 1, wl.T)
+    if wl.visibility == W.COMPRESSED:
+        return np.minimum((g + 1) // wl.ratio, wl.T)
+    return np.minimum((g + 1) // wl.ratio, wl.T // wl.ratio)
+
+
+def visible_pairs(wl, rows=None) -> int:
+    return int(visible_per_row(wl, rows).sum())
 
 
 def flops_per_pair(wl):
     return 2.0 * wl.H * wl.D
 
 
-def cpu_baseline(wl, seconds=15.0, max_rows=None):
-    """The oracle as it stands, timed on this host's cores on a bounded sample:
-    query rows at the end of the workload's query range (the rows that see the
-    most keys), drawn with the workload's shapes and distributions."""
-    import oracle
+def rank_part(wl, rank, world, scaling):
+    """(workload whose inputs this rank draws, first row, end row) of this
+    rank's share.  Strong scaling: every rank draws the whole workload (the
+    same seed: keys replicated) and takes rows [r0, r1) of the library's
+    pair-balanced split.  Weak scaling: every rank has its own problem of the
+    workload's shape (seed + 1000 * rank) and takes all of its rows."""
+    if world == 1 or scaling == "weak":
+        return (wl if world == 1 else wl.scaled(seed=wl.seed + 1000 * rank)), 0, wl.S
     from head_weighted_relu_b200 import indexer as I
-    n = 64
-    sub = wl.scaled(S=n, q_pos0=wl.q_pos0 + wl.S - n)
-    inp = W.generate(sub, "cpu")
-    prob = sub.problem()
-    hk = W.to_host_bits(inp["k"])
-    ks = W.to_host_bits(inp["k_scale"])
-    pc = W.to_host_bits(inp["pool_coef"])
-    keys = oracle.decode_keys_for(prob, hk, ks, pc)
-    done, pairs, t0 = 0, 0, time.perf_counter()
-    for t in range(n - 1, -1, -1):
-        qs = None if inp["q_scale"] is None else W.to_host_bits(inp["q_scale"][t:t + 1])
-        oracle.topk_rows(prob, W.to_host_bits(inp["q"][t:t + 1]), hk, W.to_host_bits(inp["w"][t:t + 1]),
-                         np.array([t]), q_scale_rows=qs, k_scale=ks, pool_coef=pc, keys_f64=keys)
-        pairs += I.visible_pairs(1, sub.T, sub.visibility, sub.ratio, sub.q_pos0 + t)
-        done += 1
-        if time.perf_counter() - t0 > seconds or (max_rows and done >= max_rows):
-            break
-    dt = time.perf_counter() - t0
-    try:
-        cores = len(os.sched_getaffinity(0))
-    except Exception:
-        cores = os.cpu_count()
-    return dict(value=pairs / dt / 1e9, unit="Gpairs/s", cores=cores, kind="oracle",
-                sample=f"the last {done} query rows of {wl.name} ({pairs} pairs, {dt:.1f} s); "
-                       "NumPy FP64, full score row + stable sort per row, multithreaded BLAS")
+    bounds = I.indexer_partition_rows(problem_of(wl), world)
+    return wl, bounds[rank], bounds[rank + 1]
+
+
+def problem_of(wl, r0=0, r1=None, flags=0):
+    from head_weighted_relu_b200 import indexer as I
+    r1 = wl.S if r1 is None else r1
+    return I.make_problem(r1 - r0, wl.T, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype,
+                          wl.q_pos0 + r0, flags=flags)
+
+
+def rows_of(inp, r0, r1):
+    """This rank's query rows of the inputs (keys whole)."""
+    out = dict(inp)
+    for name in ("q", "w", "q_scale"):
+        if inp[name] is not None:
+            out[name] = inp[name][r0:r1]
+    return out
+
+
+def config_of(wl, world, scaling):
+    cfg = {"workload": wl.name, "S": wl.S, "T": wl.T, "H": wl.H, "D": wl.D, "K": wl.K,
+           "visibility": ["token", "compressed", "pooled"][wl.visibility], "ratio": wl.ratio,
+           "q_pos0": wl.q_pos0, "dtype": wl.dtype, "pair_overlap": wl.pair_overlap}
+    if world > 1:
+        cfg["parallelism"] = (f"query rows split across {world} GPUs by visible-pair count, keys replicated"
+                              if scaling == "strong" else f"{world} independent problems (one per GPU)")
+    else:
+        cfg["parallelism"] = "1 GPU"
+    return cfg
+
+
+# ---------------------------------------------------------------------------
+# The CPU oracle as a baseline
+# ---------------------------------------------------------------------------
+
+def _sample_host(wl, inp, rows):
+    """Storage bits of the sampled rows (and all keys) on the host."""
+    rows_t = torch.as_tensor(rows, device=inp["q"].device)
+    sel = lambda t: None if t is None else W.to_host_bits(t.index_select(0, rows_t))  # noqa: E731
+    return dict(q=sel(inp["q"]), w=sel(inp["w"]), q_scale=sel(inp["q_scale"]),
+                k=W.to_host_bits(inp["k"]), k_scale=W.to_host_bits(inp["k_scale"]),
+                pool_coef=W.to_host_bits(inp["pool_coef"]))
+
+
+class OracleRunner:
+    """The oracle as it stands over seeded sample rows of a workload, one row
+    per host thread (NumPy's BLAS held to one thread per call)."""
+
+    def __init__(self, wl, inp, n_rows=1024):
+        import oracle
+        self.oracle = oracle
+        self.wl = wl
+        self.rows = W.sample_rows(wl, n_rows)
+        self.h = _sample_host(wl, inp, self.rows)
+        self.prob = wl.problem()
+        self.keys = oracle.decode_keys_for(self.prob, self.h["k"], self.h["k_scale"], self.h["pool_coef"])
+        self.pairs = visible_per_row(wl, self.rows)
+        try:
+            self.cores = len(os.sched_getaffinity(0))
+        except Exception:
+            self.cores = os.cpu_count() or 1
+
+    def _row(self, i):
+        h = self.h
+        self.oracle.topk_rows(self.prob, h["q"][i:i + 1], h["k"], h["w"][i:i + 1], self.rows[i:i + 1],
+                              q_scale_rows=None if h["q_scale"] is None else h["q_scale"][i:i + 1],
+                              k_scale=h["k_scale"], pool_coef=h["pool_coef"], keys_f64=self.keys)
+        return int(self.pairs[i])
+
+    def run(self, start, budget_s, threads):
+        """Rows start, start+1, ... (cyclic) until budget_s has passed;
+        returns (rows done, pairs, seconds)."""
+        from threadpoolctl import threadpool_limits
+        n = len(self.rows)
+        done = pairs = 0
+        with threadpool_limits(1):
+            t0 = time.perf_counter()
+            with cf.ThreadPoolExecutor(threads) as ex:
+                while time.perf_counter() - t0 < budget_s and done < n:
+                    batch = [(start + done + j) % n for j in range(min(threads, n - done))]
+                    pairs += sum(ex.map(self._row, batch))
+                    done += len(batch)
+            dt = time.perf_counter() - t0
+        return done, pairs, dt
+
+
+def cpu_baseline(wl, inp, all_s=12.0, one_s=6.0):
+    """The oracle timed on this host: the parity tests' 1,024 seeded query
+    rows of the workload (same inputs as the GPU run), one row per thread on
+    every core for about all_s seconds, then on one core for about one_s."""
+    r = OracleRunner(wl, inp)
+    n_all, p_all, t_all = r.run(0, all_s, r.cores)
+    n_one, p_one, t_one = r.run(0, one_s, 1)
+    v_all = p_all / t_all / 1e9
+    v_one = p_one / t_one / 1e9
+    total = visible_pairs(wl)
+    return dict(value=v_all, unit="Gpairs/s", cores=r.cores, kind="oracle",
+                one_core_value=v_one,
+                extrapolated_full_problem_s={"all_cores": total / (v_all * 1e9), "one_core": total / (v_one * 1e9),
+                                             "note": "extrapolation: the problem's pairs / the sampled rate"},
+                sample=(f"{wl.name}: the first {n_all} of the 1,024 seeded parity rows on {r.cores} threads "
+                        f"({p_all} pairs, {t_all:.1f} s), the first {n_one} on one thread ({p_one} pairs, "
+                        f"{t_one:.1f} s); NumPy FP64, full score row + stable sort per row, one row per thread"))
 
 
 def run_reference(args, wl, world, rank):
+    """The oracle as the reference arm: rank 0 only, on the machine's host cores,
+    each step a bounded sample (about 3 s) of the workload's seeded rows."""
     if rank != 0:
         return
-    base = cpu_baseline(wl, seconds=5.0)
-    steps = []
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.generate(wl, dev)          # the same seeded inputs as the GPU arm
+    r = OracleRunner(wl, inp)
+    del inp
+    start = 0
     for _ in range(args.warmup):
-        cpu_baseline(wl, seconds=2.0, max_rows=2)
+        n, _, _ = r.run(start, 0.5, r.cores)
+        start += n
+    vals, rows_done, pairs_done, secs = [], 0, 0, 0.0
     for _ in range(args.steps):
-        steps.append(cpu_baseline(wl, seconds=5.0))
-    val = statistics.median(s["value"] for s in steps)
+        n, p, dt = r.run(start, 3.0, r.cores)
+        start += n
+        vals.append(p / dt / 1e9)
+        rows_done, pairs_done, secs = rows_done + n, pairs_done + p, secs + dt
+    val = statistics.median(vals)
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": val, "unit": "Gpairs/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "Gpairs/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": args.scaling if world > 1 else "strong",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "S": wl.S, "T": wl.T, "H": wl.H, "D": wl.D, "K": wl.K},
-        "cpu_baseline": dict(base, value=val),
+        "config": config_of(wl, world, args.scaling),
+        "cpu_baseline": {"value": val, "unit": "Gpairs/s", "cores": r.cores, "kind": "oracle",
+                         "sample": f"{rows_done} of the 1,024 seeded parity rows of {wl.name} "
+                                   f"({pairs_done} pairs, {secs:.1f} s over {args.steps} steps), "
+                                   "one row per thread on every core"},
         "e2e": {"value": val, "unit": "Gpairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
 
-def planned_splits(wl, sms: int) -> int:
-    """Key-range splits the library plans for this shape (the host rule in
-    capi.cu): with fewer query blocks than half the SMs, SMs / blocks ranges of
-    at least 16 key tiles, at most 512.  A split shape adds the merge launch."""
+# ---------------------------------------------------------------------------
+# The GPU measurement
+# ---------------------------------------------------------------------------
+
+def planned_splits(wl, S, q_pos0, sms: int) -> int:
+    """Key-range splits the library plans for this shape (the host rule of
+    the C runtime): with fewer query blocks than half the SMs, SMs / blocks
+    ranges of at least 16 key tiles, at most 512.  A split shape adds the
+    merge launch."""
     qb = min(256 // wl.H, 32)
-    nb = -(-wl.S // qb)
-    if nb * 2 > sms:
+    nb = -(-S // qb)
+    if nb == 0 or nb * 2 > sms:
         return 1
-    g = wl.q_pos0 + wl.S - 1
+    g = q_pos0 + S - 1
     n_keys = wl.T // wl.ratio if wl.visibility == W.POOLED else wl.T
     nvis = min(g + 1 if wl.visibility == W.TOKEN else (g + 1) // wl.ratio, n_keys)
     s = min(sms // nb, (nvis + 127) // 128 // 16, 512)
     return s if s >= 2 else 1
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="dsa_prefill_64k", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-
-    wl = W.WORKLOADS[args.workload]
-    world, rank, local = dist_init()
-    if args.impl == "reference":
-        run_reference(args, wl, world, rank)
-        if world > 1:
-            torch.distributed.destroy_process_group()
-        return
-
+def measure(wl, inp, r0, r1, steps, warmup, dev, world, local, with_e2e=False, extras=False):
+    """Time `steps` indexer steps on rows [r0, r1) of the workload (after
+    `warmup` untimed ones), CUDA events on the launching stream, nvidia-smi
+    clocks sampled meanwhile; the time is the max over ranks."""
     from head_weighted_relu_b200 import indexer as I
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    wl_r = rank_workload(wl, rank)
-    inp = W.generate(wl_r, dev)
-    prob = I.make_problem(wl.S, wl.T, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype, wl.q_pos0)
+    mine = rows_of(inp, r0, r1)
+    S = r1 - r0
+    prob = problem_of(wl, r0, r1)
     bufs = I.allocate(prob, dev)
     stream = torch.cuda.current_stream()
-
-    # the FP8 long-context workload also counts, per non-overlapping adjacent
-    # query pair, the KV indices the two rows share (binary search)
-    shared = torch.empty((wl.S // 2,), dtype=torch.int32, device=dev) if wl.pair_overlap else None
+    shared = torch.empty((S // 2,), dtype=torch.int32, device=dev) if wl.pair_overlap else None
 
     def step():
-        I.topk(inp["q"], inp["k"], inp["w"], wl.K, visibility=wl.visibility, ratio=wl.ratio,
-               q_pos0=wl.q_pos0, q_scale=inp["q_scale"], k_scale=inp["k_scale"],
-               pool_coef=inp["pool_coef"], buffers=bufs, stream=stream)
-        if shared is not None:
-            I.indexer_pair_overlap(bufs[0], bufs[1], wl.S, bufs[0].shape[1], shared, stream)
+        if S > 0:
+            I.indexer_topk(prob, mine["q"], mine["k"], mine["w"], mine["q_scale"], mine["k_scale"],
+                           mine["pool_coef"], bufs[0], bufs[1], None, bufs[3], stream)
+            if shared is not None:
+                I.indexer_pair_overlap(bufs[0], bufs[1], S, bufs[0].shape[1], shared, stream)
 
-    for _ in range(args.warmup):
+    torch.cuda.reset_peak_memory_stats(dev)
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    status = I.indexer_read_status(bufs[3])
+    status = I.indexer_read_status(bufs[3]) if S > 0 else 0
 
-    # ---- timed region: K steps, events per step on the launching stream
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         ev[0].record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             step()
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    total_ms = max_over_ranks(total_ms, world)
-    ms_step = total_ms / args.steps
-    pairs = I.visible_pairs(wl.S, wl.T, wl.visibility, wl.ratio, wl.q_pos0)
-    value = pairs * world / (ms_step * 1e-3) / 1e9
-    peak_mem = torch.cuda.max_memory_allocated(dev) / 1e9
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world)
+    ms_step = total_ms / steps
+    pairs_all = visible_pairs(wl)          # the whole problem (strong) or one rank's (weak)
+    mine_pairs = int(visible_per_row(wl)[r0:r1].sum())
+    pk = _peaks()
+    tensor_peak = pk["bf16"] * (2.0 if wl.dtype == "fp8" else 1.0)
+    # the dominant kernel's rate on this rank's own work, from its own events
+    kern_ms = statistics.mean(per)
+    achieved = mine_pairs * flops_per_pair(wl) / (kern_ms * 1e-3) / 1e12
+    out = {
+        "ms_per_step": ms_step, "pairs_per_rank_step": mine_pairs, "pairs_per_step": pairs_all,
+        "rank_rows": [r0, r1],
+        "tensor_peak_frac": achieved / tensor_peak,
+        "peak_hbm_gb": torch.cuda.max_memory_allocated(dev) / 1e9,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tensor_peak,
+                     "peak_source": f"{pk['source']} bf16 burst" + (" x2 for fp8 (nominal ratio)" if wl.dtype == "fp8" else ""),
+                     "flops_per_pair": flops_per_pair(wl)},
+        "clocks": clk.summary(), "device_status": status,
+    }
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    splits = planned_splits(wl, S, wl.q_pos0 + r0, sms)
+    out["launches_per_step"] = (0 if S == 0 else 1 + (1 if splits > 1 else 0) + (1 if wl.visibility == W.POOLED else 0)
+                                + (1 if wl.pair_overlap else 0))
 
-    # the q-cluster preprocessing of the same pairs (shared / left-only /
-    # right-only regions), timed on its own on this step's index rows
-    regions = None
-    if shared is not None:
+    if extras and shared is not None and S >= 2:
+        # the q-cluster preprocessing of the same pairs (shared / left-only /
+        # right-only regions), timed on its own on this step's index rows
         width = bufs[0].shape[1]
-        outs = [torch.empty((wl.S // 2, width), dtype=torch.int32, device=dev) for _ in range(3)]
-        cnt = torch.empty((wl.S // 2, 3), dtype=torch.int32, device=dev)
+        outs = [torch.empty((S // 2, width), dtype=torch.int32, device=dev) for _ in range(3)]
+        cnt = torch.empty((S // 2, 3), dtype=torch.int32, device=dev)
         for _ in range(3):
-            I.indexer_pair_regions(bufs[0], bufs[1], wl.S, width, *outs, cnt, stream)
-        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        r0.record(stream)
+            I.indexer_pair_regions(bufs[0], bufs[1], S, width, *outs, cnt, stream)
+        r_0, r_1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r_0.record(stream)
         for _ in range(10):
-            I.indexer_pair_regions(bufs[0], bufs[1], wl.S, width, *outs, cnt, stream)
-        r1.record(stream)
+            I.indexer_pair_regions(bufs[0], bufs[1], S, width, *outs, cnt, stream)
+        r_1.record(stream)
         torch.cuda.synchronize()
-        r_ms = r0.elapsed_time(r1) / 10
+        r_ms = r_0.elapsed_time(r_1) / 10
         r_bytes = (bufs[0].numel() + bufs[1].numel() + 3 * outs[0].numel() + cnt.numel()) * 4
-        regions = {"ms_per_call": r_ms, "bytes_per_call": r_bytes, "gb_s": r_bytes / (r_ms * 1e-3) / 1e9}
+        out["pair_regions"] = {"ms_per_call": r_ms, "bytes_per_call": r_bytes,
+                               "gb_s": r_bytes / (r_ms * 1e-3) / 1e9}
         del outs, cnt
 
-    # decode-like shapes (few query blocks: split key ranges plus a merge) also
-    # time indexer_topk_witness, whose seed threshold shortens the per-range
-    # selection and the merge without changing the result.  Two seed sources:
-    # the same query rows' selection one decode step earlier (one key fewer;
-    # queries that change little between steps) and the row above's selection
-    # (on these i.i.d. synthetic queries it shares only chance keys).
-    splits = planned_splits(wl, torch.cuda.get_device_properties(dev).multi_processor_count)
-    witness = None
-    if splits > 1 and wl.visibility == W.TOKEN and wl.q_pos0 >= 1:
-        prev = I.make_problem(wl.S, wl.T - 1, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype, wl.q_pos0 - 1)
+    if extras and splits > 1 and wl.visibility == W.TOKEN and wl.q_pos0 + r0 >= 1:
+        # decode-like shapes also time indexer_topk_witness, whose seed
+        # threshold shortens the per-range selection and the merge without
+        # changing the result.  Seeds: the same query rows' selection one
+        # decode step earlier (one key fewer), and the row above's selection.
+        prev = I.make_problem(S, wl.T - 1, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype, wl.q_pos0 + r0 - 1)
         pb = I.allocate(prev, dev)
-        I.indexer_topk(prev, inp["q"], inp["k"], inp["w"], inp["q_scale"], inp["k_scale"], inp["pool_coef"],
+        I.indexer_topk(prev, mine["q"], mine["k"], mine["w"], mine["q_scale"], mine["k_scale"], mine["pool_coef"],
                        pb[0], pb[1], None, pb[3], stream)
         seed_sets = {"prev_step": pb[0], "row_above": torch.roll(bufs[0], 1, 0).contiguous()}
         wws = torch.empty(I.indexer_witness_workspace_bytes(prob, bufs[0].shape[1]), dtype=torch.uint8, device=dev)
@@ -304,8 +427,8 @@ def main():
             "row_above": "output row t - 1 for query row t"}}
         for name, sd in seed_sets.items():
             def wstep():
-                I.indexer_topk_witness(prob, inp["q"], inp["k"], inp["w"], inp["q_scale"], inp["k_scale"],
-                                       inp["pool_coef"], sd, w_idx, w_len, None, wws, stream)
+                I.indexer_topk_witness(prob, mine["q"], mine["k"], mine["w"], mine["q_scale"], mine["k_scale"],
+                                       mine["pool_coef"], sd, w_idx, w_len, None, wws, stream)
             for _ in range(3):
                 wstep()
             w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -317,29 +440,25 @@ def main():
             witness["ms_per_call_" + name] = w0.elapsed_time(w1) / 10
             witness["identical_" + name] = bool(torch.equal(w_idx, bufs[0]) and torch.equal(w_len, bufs[1]))
         witness["device_status"] = I.indexer_read_status(wws)
+        out["witness"] = witness
         del pb, wws, w_idx, w_len, seed_sets
 
-    pk = _peaks()
-    tensor_peak = pk["bf16"] * (2.0 if wl.dtype == "fp8" else 1.0)
-    kern_ms = statistics.mean(per)
-    achieved = pairs * flops_per_pair(wl) / (kern_ms * 1e-3) / 1e12
-
-    # ---- end to end through the C ABI with host buffers: indexer_topk_host
-    # takes page-locked host inputs and outputs; its own copies (keys once,
-    # query rows in chunks) run inside the timed region, overlapped with the
-    # indexer by the library
-    e2e = None
-    if not args.no_e2e:
-        host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+    if with_e2e:
+        # end to end through the C ABI with host buffers: indexer_topk_host
+        # takes page-locked host inputs and outputs; its own copies (keys
+        # once, query rows in chunks) run inside the timed region, overlapped
+        # with the indexer by the library
+        host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in mine.items()}
         h_idx = torch.empty(bufs[0].shape, dtype=torch.int32).pin_memory()
         h_len = torch.empty(bufs[1].shape, dtype=torch.int32).pin_memory()
-        hws = torch.empty(I.indexer_host_workspace_bytes(prob), dtype=torch.uint8, device=dev)
+        hws = torch.empty(max(I.indexer_host_workspace_bytes(prob), 256), dtype=torch.uint8, device=dev)
         h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
         d2h = h_idx.numel() * 4 + h_len.numel() * 4
 
         def e2e_step():
-            I.indexer_topk_host(prob, host["q"], host["k"], host["w"], host["q_scale"], host["k_scale"],
-                                host["pool_coef"], h_idx, h_len, None, hws, stream)
+            if S > 0:
+                I.indexer_topk_host(prob, host["q"], host["k"], host["w"], host["q_scale"], host["k_scale"],
+                                    host["pool_coef"], h_idx, h_len, None, hws, stream)
 
         for _ in range(2):
             e2e_step()
@@ -347,22 +466,81 @@ def main():
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        n_e2e = max(1, min(args.steps, 5))
+        n_e2e = max(1, min(steps, 5))
         for _ in range(n_e2e):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
-        e2e = {"value": pairs * world / (e2e_ms * 1e-3) / 1e9, "unit": "Gpairs/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "api": "indexer_topk_host (pinned host buffers, copies overlapped with the indexer)"}
+        out["e2e"] = {"value": None, "unit": "Gpairs/s", "ms_per_step": e2e_ms,
+                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                      "api": "indexer_topk_host (pinned host buffers, copies overlapped with the indexer)"}
         if shared is not None:
-            e2e["excludes"] = "the pair-overlap count (it runs on the device rows of the indexer_topk step)"
+            out["e2e"]["excludes"] = "the pair-overlap count (it runs on the device rows of the indexer_topk step)"
         del host, hws
+    del bufs
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dsa_prefill_64k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--scaling", default="strong", choices=["strong", "weak"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration map")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    wl = W.WORKLOADS[args.workload]
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    gen_wl, r0, r1 = rank_part(wl, rank, world, args.scaling)
+    inp = W.generate(gen_wl, dev)
+    res = measure(gen_wl, inp, r0, r1, args.steps, args.warmup, dev, world, local,
+                  with_e2e=not args.no_e2e, extras=True)
+    strong = world > 1 and args.scaling == "strong"
+    total_pairs = res["pairs_per_step"] * (1 if strong or world == 1 else world)
+    value = total_pairs / (res["ms_per_step"] * 1e-3) / 1e9
+    if res.get("e2e"):
+        res["e2e"]["value"] = total_pairs / (res["e2e"]["ms_per_step"] * 1e-3) / 1e9
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        base = cpu_baseline(wl)
+        base = cpu_baseline(wl, inp)
+    del inp
+    torch.cuda.empty_cache()
+
+    # every configuration the metric is quoted on, measured the same way
+    # (fewer steps, no end-to-end leg) at N = 1
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = {}
+        for name in QUOTED_CONFIGS:
+            cw = W.WORKLOADS[name]
+            if name == wl.name:
+                r = res
+            else:
+                cin = W.generate(cw, dev)
+                r = measure(cw, cin, 0, cw.S, min(args.steps, 5), 3, dev, 1, local)
+                del cin
+                torch.cuda.empty_cache()
+            configs[name] = {"value": r["pairs_per_step"] / (r["ms_per_step"] * 1e-3) / 1e9, "unit": "Gpairs/s",
+                             "ms_per_step": r["ms_per_step"], "roofline_frac": r["roofline"]["frac"],
+                             "tensor_peak": r["roofline"]["peak_source"], "peak_hbm_gb": r["peak_hbm_gb"],
+                             "queries_per_s": cw.S / (r["ms_per_step"] * 1e-3), "clocks": r["clocks"],
+                             "device_status": r["device_status"], "steps": min(args.steps, 5) if name != wl.name else args.steps}
 
     traffic = None
     try:
@@ -371,35 +549,29 @@ def main():
     except Exception:
         traffic = None
 
-    launches_per_step = (1 + (1 if splits > 1 else 0) + (1 if wl.visibility == W.POOLED else 0)
-                         + (1 if wl.pair_overlap else 0))
     if rank == 0:
+        roof = dict(res["roofline"], traffic=traffic)
         out = {
             "metric": METRIC, "value": value, "unit": "Gpairs/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+            "higher_is_better": True, "scaling": args.scaling if world > 1 else "strong",
+            "vs_baseline": None,
             "dtype": "fp8-e4m3 (fp32 accumulate)" if wl.dtype == "fp8" else "bf16 (fp32 accumulate)",
             "data": "synthetic",
-            "config": {"workload": wl.name, "S": wl.S, "T": wl.T, "H": wl.H, "D": wl.D, "K": wl.K,
-                       "visibility": ["token", "compressed", "pooled"][wl.visibility], "ratio": wl.ratio,
-                       "q_pos0": wl.q_pos0, "pair_overlap": wl.pair_overlap,
-                       "parallelism": f"{world} independent problems (one per GPU)",
-                       "l2": "inputs larger than L2 (q alone is "
-                             f"{inp['q'].numel() * inp['q'].element_size() / 2**30:.2f} GiB)"},
-            "pairs_per_step": pairs, "queries_per_s": wl.S * world / (ms_step * 1e-3),
-            "tensor_peak_frac": achieved / tensor_peak,
-            "peak_hbm_gb": peak_mem,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                         "frac": achieved / tensor_peak, "traffic": traffic,
-                         "peak_source": f"{pk['source']} bf16 burst" + (" x2 for fp8 (nominal ratio)" if wl.dtype == "fp8" else ""),
-                         "flops_per_pair": flops_per_pair(wl)},
-            "clocks": clk.summary(),
-            "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
-            "pair_regions": regions,
-            "witness": witness,
-            "device_status": status,
+            "config": dict(config_of(wl, world, args.scaling),
+                           l2=f"inputs larger than L2 (q alone is {wl.S * wl.H * wl.D * (1 if wl.dtype == 'fp8' else 2) / 2**30:.2f} GiB)"),
+            "pairs_per_step": total_pairs, "queries_per_s": wl.S * (1 if strong or world == 1 else world) / (res["ms_per_step"] * 1e-3),
+            "tensor_peak_frac": res["tensor_peak_frac"],
+            "peak_hbm_gb": res["peak_hbm_gb"],
+            "roofline": roof,
+            "clocks": res["clocks"],
+            "e2e": res.get("e2e"),
+            "gpu_launches": res["launches_per_step"] * args.steps,
+            "pair_regions": res.get("pair_regions"),
+            "witness": res.get("witness"),
+            "device_status": res["device_status"],
             "cpu_baseline": base,
+            "configs": configs,
         }
         print(json.dumps(out))
     if world > 1:

@@ -212,6 +212,46 @@ indexer_status indexer_workspace_bytes(const indexer_problem* p, size_t* bytes) 
   return INDEXER_OK;
 }
 
+indexer_status indexer_partition_rows(const indexer_problem* p, int32_t n_parts, int64_t* bounds) {
+  Plan pl;
+  const indexer_status st = make_plan(p, false, &pl);
+  if (st != INDEXER_OK) return st;
+  if (!bounds || n_parts < 1 || n_parts > 4096) return INDEXER_EINVAL;
+  // visible keys (pools) of row t; rows are independent problems, and the
+  // scoring work of a row is its visible count
+  const int64_t ratio = pl.ranged ? p->ratio : 1;
+  auto visible = [&](int64_t t) -> int64_t {
+    const int64_t g = p->q_pos0 + t;
+    const int64_t n = pl.ranged ? (g + 1) / ratio : g + 1;
+    return n < pl.n_keys ? n : pl.n_keys;
+  };
+  const int64_t qb = pl.var.queries_per_block;
+  const int64_t n_blocks = (p->S + qb - 1) / qb;
+  int64_t total = 0;
+  for (int64_t t = 0; t < p->S; ++t) total += visible(t);
+  // cut i goes to the query-block boundary whose pair prefix is nearest to
+  // i * total / n_parts (each part then differs from an equal share by at
+  // most one block's pairs)
+  bounds[0] = 0;
+  int64_t blk = 0, prefix = 0;  // pairs of rows [0, blk * qb)
+  for (int32_t i = 1; i < n_parts; ++i) {
+    const long double target = static_cast<long double>(total) * i / n_parts;
+    while (blk < n_blocks) {
+      int64_t bp = 0;
+      const int64_t r1 = (blk + 1) * qb < p->S ? (blk + 1) * qb : p->S;
+      for (int64_t t = blk * qb; t < r1; ++t) bp += visible(t);
+      // advance while the boundary after this block is nearer the target
+      if (static_cast<long double>(prefix) + bp / 2.0L > target) break;
+      prefix += bp;
+      ++blk;
+    }
+    const int64_t r = blk * qb < p->S ? blk * qb : p->S;
+    bounds[i] = r > bounds[i - 1] ? r : bounds[i - 1];
+  }
+  bounds[n_parts] = p->S;
+  return INDEXER_OK;
+}
+
 }  // extern "C"
 
 namespace hwr {
@@ -725,6 +765,124 @@ indexer_status indexer_docs_workspace_bytes(const indexer_problem* p, const int6
     most = b > most ? b : most;
   }
   *bytes = most > 256 ? most : 256;
+  return INDEXER_OK;
+}
+
+}  // extern "C"
+
+namespace hwr {
+namespace {
+
+// Sequence b of a padded batch as an indexer problem of its own: rows
+// [b*stride, b*stride + len), positions from 0, keys from its first row.
+// `empty` when it has no query row or (compressed keys) no complete key.
+indexer_status seq_part(const indexer_problem* p, const int64_t* lens, int64_t stride, int32_t b, DocPart* out,
+                        bool* empty) {
+  const bool compressed = p->visibility == INDEXER_VIS_COMPRESSED;
+  const int64_t ratio = p->visibility == INDEXER_VIS_TOKEN ? 1 : p->ratio;
+  out->sub = *p;
+  out->sub.S = lens[b];
+  out->sub.q_pos0 = 0;
+  out->sub.T = compressed ? lens[b] / ratio : lens[b];
+  out->r0 = b * stride;
+  out->key0 = compressed ? b * stride / ratio : b * stride;
+  if (out->key0 > INT32_MAX) return INDEXER_EUNSUPPORTED;
+  out->shift = static_cast<int32_t>(out->key0);
+  *empty = out->sub.S == 0 || out->sub.T == 0;
+  return INDEXER_OK;
+}
+
+// S and T cover every padded row, q_pos0 is 0, lengths fit their stride, and
+// (compressed keys) the stride is a whole number of compressed keys.
+indexer_status check_padded(const indexer_problem* p, const int64_t* lens, int32_t n_seqs, int64_t stride) {
+  if (!p || !lens || n_seqs < 1 || stride < 1) return INDEXER_EINVAL;
+  const bool compressed = p->visibility == INDEXER_VIS_COMPRESSED;
+  const int64_t ratio = p->visibility == INDEXER_VIS_TOKEN ? 1 : p->ratio;
+  if (ratio < 1 || (compressed && stride % ratio != 0)) return INDEXER_EINVAL;
+  if (p->q_pos0 != 0 || p->S != n_seqs * stride) return INDEXER_EINVAL;
+  if (p->T != (compressed ? n_seqs * stride / ratio : n_seqs * stride)) return INDEXER_EINVAL;
+  for (int32_t b = 0; b < n_seqs; ++b)
+    if (lens[b] < 0 || lens[b] > stride) return INDEXER_EINVAL;
+  return INDEXER_OK;
+}
+
+}  // namespace
+}  // namespace hwr
+
+extern "C" {
+
+indexer_status indexer_padded_workspace_bytes(const indexer_problem* p, const int64_t* seq_lens, int32_t n_seqs,
+                                              int64_t stride, size_t* bytes) {
+  indexer_status st = check_padded(p, seq_lens, n_seqs, stride);
+  if (st != INDEXER_OK) return st;
+  if (!bytes) return INDEXER_EINVAL;
+  size_t most = 0;
+  for (int32_t b = 0; b < n_seqs; ++b) {
+    DocPart part;
+    bool empty = false;
+    st = seq_part(p, seq_lens, stride, b, &part, &empty);
+    if (st != INDEXER_OK) return st;
+    if (empty) continue;
+    size_t need = 0;
+    st = indexer_workspace_bytes(&part.sub, &need);
+    if (st != INDEXER_OK) return st;
+    most = need > most ? need : most;
+  }
+  *bytes = most > 256 ? most : 256;
+  return INDEXER_OK;
+}
+
+indexer_status indexer_topk_padded(const indexer_problem* p, const void* q, const void* k, const float* w,
+                                   const float* q_scale, const float* k_scale, const void* pool_coef,
+                                   const int64_t* seq_lens, int32_t n_seqs, int64_t stride, int32_t* out_idx,
+                                   int32_t* out_len, float* out_score, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  indexer_status st = check_padded(p, seq_lens, n_seqs, stride);
+  if (st != INDEXER_OK) return st;
+  if (!q || !k || !w || !out_idx || !out_len) return INDEXER_EINVAL;
+  if (p->dtype == INDEXER_FP8_E4M3 && (!q_scale || !k_scale)) return INDEXER_EINVAL;
+  if (p->visibility == INDEXER_VIS_POOLED && !pool_coef) return INDEXER_EINVAL;
+  size_t need = 0;
+  st = indexer_padded_workspace_bytes(p, seq_lens, n_seqs, stride, &need);
+  if (st != INDEXER_OK) return st;
+  if (!workspace || !aligned(workspace, 256)) return INDEXER_EWORKSPACE;
+  if (workspace_bytes < need) return INDEXER_EWORKSPACE;
+  const size_t elem = p->dtype == INDEXER_FP8_E4M3 ? 1 : 2;
+  int32_t width = 0;
+  st = indexer_out_width(p, &width);
+  if (st != INDEXER_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status word and counters start at zero once for all sequences
+  if (cudaMemsetAsync(workspace, 0, 32, s) != cudaSuccess) return INDEXER_ECUDA;
+  const size_t q_row = static_cast<size_t>(p->H) * p->D * elem;
+  for (int32_t b = 0; b < n_seqs; ++b) {
+    DocPart part;
+    bool empty = false;
+    st = seq_part(p, seq_lens, stride, b, &part, &empty);
+    if (st != INDEXER_OK) return st;
+    // rows that select nothing: the sequence's padding, and every row of a
+    // sequence without a visible key (length 0, indices -1, scores NaN)
+    const int64_t first_empty = empty ? part.r0 : part.r0 + part.sub.S;
+    const int64_t n_empty = part.r0 + stride - first_empty;
+    if (n_empty > 0) {
+      if (cudaMemsetAsync(out_idx + first_empty * width, 0xFF, n_empty * width * sizeof(int32_t), s) != cudaSuccess ||
+          cudaMemsetAsync(out_len + first_empty, 0, n_empty * sizeof(int32_t), s) != cudaSuccess ||
+          (out_score && cudaMemsetAsync(out_score + first_empty * width, 0xFF, n_empty * width * sizeof(float), s) !=
+                            cudaSuccess))
+        return INDEXER_ECUDA;
+    }
+    if (empty) continue;
+    const int64_t r0 = part.r0;
+    st = run_topk(&part.sub, static_cast<const uint8_t*>(q) + r0 * q_row,
+                  static_cast<const uint8_t*>(k) + part.key0 * static_cast<int64_t>(p->D) * elem, w + r0 * p->H,
+                  q_scale ? q_scale + r0 * p->H : nullptr, k_scale ? k_scale + part.key0 : nullptr, pool_coef,
+                  out_idx + r0 * width, out_len + r0, out_score ? out_score + r0 * width : nullptr, workspace,
+                  workspace_bytes, stream, false);
+    if (st != INDEXER_OK) return st;
+    if (part.shift != 0 &&
+        launch_offset_indices(out_idx + r0 * width, part.sub.S * width, part.shift, s) != cudaSuccess)
+      return INDEXER_ECUDA;
+  }
   return INDEXER_OK;
 }
 

@@ -26,7 +26,8 @@ void* g_scratch_addr[kMaxDevices];
 std::mutex g_scratch_mutex;
 
 // Device address of the scratch array on the current device; looked up on
-// the first call per device (with that device current) and cached.
+// the first call per device (with that device current) and cached for the
+// life of the process (a cudaDeviceReset would invalidate it).
 indexer_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return INDEXER_ECUDA;
@@ -56,6 +57,16 @@ indexer_status indexer_topk_noalloc(const indexer_problem* p, const void* q, con
   if (st != INDEXER_OK) return st;
   return indexer_topk(p, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len, out_score, scratch,
                       kNoAllocScratchBytes, stream);
+}
+
+indexer_status indexer_noalloc_read_status(int32_t* flags, void* stream) {
+  if (!flags) return INDEXER_EINVAL;
+  void* scratch = nullptr;
+  indexer_status st = scratch_address(&scratch);
+  if (st != INDEXER_OK) return st;
+  // the status word sits at the start of the scratch array, as at the start
+  // of any indexer_topk workspace
+  return indexer_read_status(scratch, flags, stream);
 }
 
 }  // extern "C"

@@ -29,14 +29,16 @@ STATUS_NAMES = {0: "INDEXER_OK", 1: "INDEXER_EINVAL", 2: "INDEXER_EWORKSPACE",
                 3: "INDEXER_EUNSUPPORTED", 4: "INDEXER_ECUDA", 5: "INDEXER_EDEVICE"}
 
 # every symbol include/hwr_indexer.h declares
-EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_topk", "indexer_topk_noalloc",
+EXPORTS = ("indexer_out_width", "indexer_workspace_bytes", "indexer_partition_rows",
+           "indexer_topk", "indexer_topk_noalloc", "indexer_noalloc_read_status",
            "indexer_host_workspace_bytes", "indexer_topk_host",
            "indexer_docs_workspace_bytes", "indexer_topk_docs",
+           "indexer_padded_workspace_bytes", "indexer_topk_padded",
            "indexer_witness_workspace_bytes", "indexer_topk_witness",
            "indexer_pool_keys",
            "indexer_pair_overlap", "indexer_pair_regions", "indexer_read_status", "indexer_read_prune_counters",
            "indexer_status_string",
-           "indexer_abi_version")
+           "indexer_abi_version", "indexer_build_info")
 
 
 class IndexerError(RuntimeError):
@@ -60,16 +62,32 @@ def _load():
             f"{LIB_PATH} is missing: build it with `python -m head_weighted_relu_b200.build` "
             "(the indexer has no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
+    lib.indexer_build_info.argtypes = []
+    lib.indexer_build_info.restype = ctypes.c_char_p
+    if "HWR_INDEXER_LIB" not in os.environ:
+        # the library must come from the sources beside it (a stale build would
+        # otherwise pass unnoticed)
+        from . import build as _build
+        want = "source_sha256=" + _build.source_hash()
+        got = lib.indexer_build_info().decode()
+        if got != want:
+            raise ImportError(f"{LIB_PATH} was built from other sources ({got[:30]}...); "
+                              "rebuild it with `python -m head_weighted_relu_b200.build`")
     P = ctypes.POINTER(Problem)
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     lib.indexer_out_width.argtypes = [P, ctypes.POINTER(i32)]
     lib.indexer_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+    lib.indexer_partition_rows.argtypes = [P, i32, ctypes.POINTER(i64)]
     lib.indexer_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.indexer_noalloc_read_status.argtypes = [ctypes.POINTER(i32), vp]
     lib.indexer_host_workspace_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
     lib.indexer_topk_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_docs_workspace_bytes.argtypes = [P, vp, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.indexer_topk_docs.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.indexer_padded_workspace_bytes.argtypes = [P, vp, i32, i64, ctypes.POINTER(ctypes.c_size_t)]
+    lib.indexer_topk_padded.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp,
+                                        ctypes.c_size_t, vp]
     lib.indexer_witness_workspace_bytes.argtypes = [P, i64, ctypes.POINTER(ctypes.c_size_t)]
     lib.indexer_topk_witness.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.indexer_pool_keys.argtypes = [vp, i64, i32, vp, i32, vp, vp]
@@ -81,7 +99,7 @@ def _load():
     lib.indexer_status_string.restype = ctypes.c_char_p
     lib.indexer_abi_version.argtypes = []
     for name in EXPORTS:
-        if name not in ("indexer_status_string",):
+        if name not in ("indexer_status_string", "indexer_build_info"):
             getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -123,6 +141,14 @@ def indexer_workspace_bytes(problem: Problem) -> int:
     _check("indexer_workspace_bytes",
            _lib.indexer_workspace_bytes(ctypes.byref(problem), ctypes.byref(n)))
     return n.value
+
+
+def indexer_partition_rows(problem: Problem, n_parts: int) -> list:
+    """Row bounds [0, ..., S] splitting the problem's query rows into n_parts
+    parts of about equal visible-pair count (one part per GPU)."""
+    b = (ctypes.c_int64 * (n_parts + 1))()
+    _check("indexer_partition_rows", _lib.indexer_partition_rows(ctypes.byref(problem), n_parts, b))
+    return [int(x) for x in b]
 
 
 def indexer_topk(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len, out_score,
@@ -198,6 +224,26 @@ def indexer_topk_docs(problem, q, k, w, q_scale, k_scale, pool_coef, doc_bounds,
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def indexer_padded_workspace_bytes(problem: Problem, seq_lens, stride: int) -> int:
+    b, ptr, n = _bounds(seq_lens)
+    out = ctypes.c_size_t()
+    _check("indexer_padded_workspace_bytes",
+           _lib.indexer_padded_workspace_bytes(ctypes.byref(problem), ptr, n + 1, stride, ctypes.byref(out)))
+    return out.value
+
+
+def indexer_topk_padded(problem, q, k, w, q_scale, k_scale, pool_coef, seq_lens, stride, out_idx, out_len,
+                        out_score, workspace, stream=None):
+    """indexer_topk for a padded batch: sequence b is rows b*stride ..
+    b*stride + seq_lens[b] - 1 (seq_lens on the host); padding rows select
+    nothing."""
+    b, ptr, n = _bounds(seq_lens)
+    _check("indexer_topk_padded", _lib.indexer_topk_padded(
+        ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale), _ptr(pool_coef),
+        ptr, n + 1, stride, _ptr(out_idx), _ptr(out_len), _ptr(out_score), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def indexer_topk_noalloc(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx, out_len,
                          out_score, stream=None):
     """indexer_topk without a workspace: for callers that cannot allocate device
@@ -207,6 +253,13 @@ def indexer_topk_noalloc(problem, q, k, w, q_scale, k_scale, pool_coef, out_idx,
     _check("indexer_topk_noalloc", _lib.indexer_topk_noalloc(
         ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(w), _ptr(q_scale), _ptr(k_scale),
         _ptr(pool_coef), _ptr(out_idx), _ptr(out_len), _ptr(out_score), _stream(stream)))
+
+
+def indexer_noalloc_read_status(stream=None) -> int:
+    """Status word of the last indexer_topk_noalloc call (read and cleared)."""
+    f = ctypes.c_int32()
+    _check("indexer_noalloc_read_status", _lib.indexer_noalloc_read_status(ctypes.byref(f), _stream(stream)))
+    return f.value
 
 
 def indexer_pool_keys(k, T_tokens, D, pool_coef, ratio, out_kp, stream=None):
@@ -243,6 +296,11 @@ def indexer_read_prune_counters(workspace, stream=None):
 
 def indexer_abi_version() -> int:
     return _lib.indexer_abi_version()
+
+
+def indexer_build_info() -> str:
+    """The build's identity: "source_sha256=<hash of the sources and flags>"."""
+    return _lib.indexer_build_info().decode()
 
 
 # ---------------------------------------------------------------------------
@@ -318,17 +376,3 @@ def pool_keys(k, pool_coef, ratio, stream=None):
     out = torch.empty((T // ratio, D), dtype=torch.bfloat16, device=k.device)
     indexer_pool_keys(k.contiguous(), T, D, pool_coef.contiguous(), ratio, out, stream)
     return out
-
-
-def visible_pairs(S, T, visibility=TOKEN, ratio=1, q_pos0=0) -> int:
-    """Number of (query, key) pairs the indexer scores: for each query at
-    global position g, the keys visible to it (pools for POOLED)."""
-    import numpy as np
-    g = np.arange(S, dtype=np.int64) + q_pos0
-    if visibility == TOKEN:
-        n = np.minimum(g + 1, T)
-    elif visibility == COMPRESSED:
-        n = np.minimum((g + 1) // ratio, T)
-    else:
-        n = np.minimum((g + 1) // ratio, T // ratio)
-    return int(n.sum())

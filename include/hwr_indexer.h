@@ -120,6 +120,21 @@ indexer_status indexer_out_width(const indexer_problem* p, int32_t* width);
  * except the status words read by indexer_read_status. */
 indexer_status indexer_workspace_bytes(const indexer_problem* p, size_t* bytes);
 
+/* Split of one problem's query rows across n_parts devices (one process per
+ * GPU, keys replicated on every device): writes bounds[0 .. n_parts] (HOST
+ * array) with bounds[0] = 0, bounds[n_parts] = S, non-decreasing, every bound
+ * a multiple of the compiled variant's query block (or S).  Part i is rows
+ * [bounds[i], bounds[i+1]): an indexer problem of its own with S' = its row
+ * count and q_pos0' = q_pos0 + bounds[i], reading rows bounds[i].. of q, w
+ * and q_scale and writing the same rows of the outputs.  Rows are
+ * independent, so the parts need no exchange; cuts are placed by visible
+ * (query, key) pair count, not by row count, since under causal visibility
+ * later rows see more keys: each part's pair count is within one query
+ * block's pairs of an equal share.  Pure host computation (no device call);
+ * INDEXER_EINVAL for an invalid problem, n_parts < 1 or > 4096, or a null
+ * `bounds`. */
+indexer_status indexer_partition_rows(const indexer_problem* p, int32_t n_parts, int64_t* bounds);
+
 /* The indexer: scores, top-K and finalisation in one call.
  *   q         [S, H, D]  bf16, or e4m3 codes (uint8) for INDEXER_FP8_E4M3
  *   k         [T, D]     same storage as q
@@ -164,14 +179,21 @@ indexer_status indexer_topk(const indexer_problem* p,
  *   previous call's contents (each call clears what must start at zero), so
  *   calls that may overlap on the GPU -- on different streams, or from
  *   different host threads -- race and corrupt each other's results;
- *   serialise them.  indexer_read_status does not apply to this entry point
- *   (there is no workspace to pass it). */
+ *   serialise them.  The device status word of a call (see indexer_read_status)
+ *   is read with indexer_noalloc_read_status.  The array's device address is
+ *   cached per device for the life of the process; after a cudaDeviceReset
+ *   of that device the entry point must not be used again. */
 indexer_status indexer_topk_noalloc(const indexer_problem* p,
                                     const void* q, const void* k, const float* w,
                                     const float* q_scale, const float* k_scale,
                                     const void* pool_coef,
                                     int32_t* out_idx, int32_t* out_len, float* out_score,
                                     void* stream);
+
+/* indexer_read_status for indexer_topk_noalloc: synchronises `stream`, reads
+ * and clears the status word kept at the start of the fixed scratch array
+ * (the same bits as indexer_read_status).  Allocates nothing. */
+indexer_status indexer_noalloc_read_status(int32_t* flags, void* stream);
 
 /* indexer_topk on HOST buffers (page-locked for the copies to overlap):
  * q, k, w, q_scale, k_scale and pool_coef are host pointers with the layouts
@@ -264,6 +286,32 @@ indexer_status indexer_topk_docs(const indexer_problem* p, const void* q, const 
                                  int32_t* out_idx, int32_t* out_len, float* out_score,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* indexer_topk for a padded batch ("Module 06 — DSA & KPool", §3 and "Ship
+ * it": the boundary lengths are checked with and without padding, and a
+ * padding position must never reach a selection).  The batch holds n_seqs
+ * sequences, each padded to `stride` rows: sequence b is query rows and token
+ * keys b*stride .. b*stride + seq_lens[b] - 1, and the rest of its stride is
+ * padding.  seq_lens is a HOST array (0 <= seq_lens[b] <= stride).
+ *   p->S = n_seqs*stride query rows, p->q_pos0 = 0, p->T = n_seqs*stride
+ *   token keys (TOKEN, POOLED) or n_seqs*stride/ratio compressed keys
+ *   (COMPRESSED; stride a multiple of the ratio).
+ * Inside a sequence everything is as for a sequence of its own, positions
+ * counted from its first row (pools form from its first token, its own
+ * incomplete tail is appended); output indices are rows of the padded key
+ * array.  Padding query rows -- and rows that see no key -- get length 0,
+ * indices -1 and scores NaN.  Workspace: indexer_padded_workspace_bytes
+ * bytes; indexer_read_status covers every sequence.  Each sequence runs as
+ * its own indexer call on `stream`.  Errors as indexer_topk, INDEXER_EINVAL
+ * for sizes that do not fit the rules above. */
+indexer_status indexer_padded_workspace_bytes(const indexer_problem* p, const int64_t* seq_lens,
+                                              int32_t n_seqs, int64_t stride, size_t* bytes);
+indexer_status indexer_topk_padded(const indexer_problem* p, const void* q, const void* k,
+                                   const float* w, const float* q_scale,
+                                   const float* k_scale, const void* pool_coef,
+                                   const int64_t* seq_lens, int32_t n_seqs, int64_t stride,
+                                   int32_t* out_idx, int32_t* out_len, float* out_score,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* Pool formation alone (the first step of POOLED):
  *   kp[p, d] = RNE_bf16( exact sum_{j<ratio} c[j, d] * k[ratio*p + j, d] )
  * for p < T_tokens / ratio; k [T_tokens, D] bf16, pool_coef [ratio, D] bf16,
@@ -325,6 +373,10 @@ const char* indexer_status_string(indexer_status s);
 
 /* Version of this ABI (incremented on incompatible change). */
 int32_t indexer_abi_version(void);
+
+/* Identity of this build: "source_sha256=" and the SHA-256 of the sources and
+ * compile flags it was built from (static storage). */
+const char* indexer_build_info(void);
 
 #ifdef __cplusplus
 }

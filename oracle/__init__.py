@@ -26,6 +26,7 @@ from .indexer_oracle import (  # noqa: F401
     out_width,
     topk_rows,
     topk_rows_docs,
+    topk_rows_padded,
     witness_seed_keys,
     witness_threshold,
     decode_keys_for,

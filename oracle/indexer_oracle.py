@@ -449,6 +449,83 @@ def topk_rows_docs(problem: dict, q_rows, k, w_rows, rows, doc_bounds, q_scale_r
     return out_idx, out_len, out_score, taus
 
 
+def topk_rows_padded(problem: dict, q_rows, k, w_rows, rows, seq_lens, stride: int,
+                     q_scale_rows=None, k_scale=None, pool_coef=None):
+    """Indexer output for query rows of a padded batch.
+
+    The batch holds len(seq_lens) sequences, each padded to `stride` token
+    rows: sequence b occupies rows b*stride .. b*stride + seq_lens[b] - 1 of
+    the queries and of the token keys, and the rest of its stride is padding.
+    A padding position is never visible and a padding query row selects
+    nothing (length 0, all -1).  Inside a sequence everything is as for one
+    sequence of its own ("Module 06 — DSA & KPool: Selective Retrieval", §3
+    and "Ship it": every watch length checked with and without padding), with
+    positions relative to the sequence start: the query at position j of
+    sequence b sees
+      TOKEN       token keys b*stride .. b*stride + j;
+      COMPRESSED  compressed keys b*stride/ratio + c with ratio*c+ratio-1 <= j
+                  (stride a multiple of the ratio);
+      POOLED      the sequence's pools, pool c formed from tokens
+                  b*stride + ratio*c .. + ratio-1, visible once complete, then
+                  the tail b*stride + ratio*nc .. b*stride + j.
+    Indices are rows of the padded key array.  Arguments and results as
+    topk_rows (problem["S"] = number of query rows of the padded batch).
+    """
+    vis_mode = problem["visibility"]
+    ratio = int(problem["ratio"]) if vis_mode != TOKEN else 1
+    K = int(problem["K"])
+    width = out_width(K, vis_mode, ratio)
+    ksel = K // ratio if vis_mode == POOLED else K
+    R = len(rows)
+    out_idx = np.full((R, width), -1, dtype=np.int32)
+    out_len = np.zeros(R, dtype=np.int32)
+    out_score = np.full((R, width), math.nan, dtype=np.float64)
+    taus = np.full(R, math.nan, dtype=np.float64)
+    tokens = None if vis_mode == POOLED else _decode_keys(problem, k, k_scale, pool_coef)
+    pooled_cache = {}
+    for r in range(R):
+        t = int(rows[r])
+        b, j = divmod(t, stride)
+        if j >= int(seq_lens[b]):
+            continue                                  # a padding query row
+        start = b * stride
+        if problem["dtype"] == "fp8":
+            q_t = decode_e4m3(q_rows[r]) * np.asarray(q_scale_rows[r], dtype=np.float64)[:, None]
+        else:
+            q_t = decode_bf16(q_rows[r])
+        w_t = np.asarray(w_rows[r], dtype=np.float64)
+        if vis_mode == TOKEN:
+            vis = np.arange(start, start + j + 1, dtype=np.int64)
+            block = tokens[vis]
+        elif vis_mode == COMPRESSED:
+            c = np.arange((j + 1) // ratio, dtype=np.int64)      # complete compressed keys so far
+            vis = start // ratio + c
+            block = tokens[vis]
+        else:
+            if b not in pooled_cache:
+                n_tok = int(seq_lens[b])
+                pooled_cache[b] = decode_bf16(pooled_keys(np.asarray(k)[start:start + n_tok], pool_coef, ratio))
+            n_done = (j + 1) // ratio
+            vis = np.arange(n_done, dtype=np.int64)              # sequence-local pool numbers
+            block = pooled_cache[b][:n_done]
+        s = score_keys(q_t, w_t, block)
+        sel, ssel, tau = select_topk(s, vis, ksel)
+        taus[r] = tau
+        if vis_mode == POOLED:
+            pos = (start + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)
+            sc = np.repeat(ssel, ratio)
+            tail = np.arange(start + ratio * n_done, start + j + 1, dtype=np.int64)
+            pos = np.concatenate((pos, tail))
+            sc = np.concatenate((sc, np.full(tail.size, math.nan)))
+        else:
+            pos, sc = sel, ssel
+        n = pos.size
+        out_idx[r, :n] = pos
+        out_len[r] = n
+        out_score[r, :n] = sc
+    return out_idx, out_len, out_score, taus
+
+
 def decode_keys_for(problem: dict, k, k_scale=None, pool_coef=None) -> np.ndarray:
     """Decoded float64 keys (pooled keys for POOLED) for reuse across calls."""
     return _decode_keys(problem, k, k_scale, pool_coef)

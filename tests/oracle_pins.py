@@ -609,6 +609,48 @@ def pin_documents_compressed(O):
             assert ln[t] == 0, t
 
 
+def pin_padded_batch(O):
+    """Padded batches ("Module 06 — DSA & KPool", §3 and "Ship it": the watch
+    lengths 3, 4, 5, 7, 8, 9 checked with and without padding): every real
+    row of a padded batch equals the plain indexer run on its sequence alone
+    (sliced out, positions from 0), shifted by the sequence's first row;
+    padding rows select nothing; with no padding the batch equals a packed
+    batch whose documents start at multiples of the stride."""
+    rng = np.random.default_rng(47)
+    H, D, stride = 3, 8, 12
+    lens = [3, 4, 5, 7, 8, 9]
+    n = stride * len(lens)
+    qb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(n, H, D)))
+    kb = _bf16_bits_of_ints(rng.integers(-3, 4, size=(n, D)))
+    w = rng.integers(-2, 3, size=(n, H)).astype(np.float32)
+    rows = np.arange(n)
+    for vis, ratio, K in ((O.TOKEN, 1, 4), (O.COMPRESSED, 4, 2), (O.POOLED, 4, 4)):
+        c = _bf16_bits_of_ints(rng.integers(0, 3, size=(ratio, D))) if vis == O.POOLED else None
+        keys_all = kb if vis != O.COMPRESSED else kb[: n // ratio]
+        prob = _problem(S=n, T=keys_all.shape[0], H=H, D=D, K=K, vis=vis, ratio=ratio)
+        idx, ln, _, _ = O.topk_rows_padded(prob, qb, keys_all, w, rows, lens, stride, pool_coef=c)
+        for b, L in enumerate(lens):
+            r0 = b * stride
+            assert (ln[r0 + L: r0 + stride] == 0).all() and (idx[r0 + L: r0 + stride] == -1).all(), (vis, b)
+            if vis == O.COMPRESSED:
+                kk, shift = kb[r0 // ratio: (r0 + L) // ratio], r0 // ratio
+                if kk.shape[0] == 0:
+                    assert (ln[r0: r0 + L] == 0).all()
+                    continue
+            else:
+                kk, shift = kb[r0: r0 + L], r0
+            one = _problem(S=L, T=kk.shape[0], H=H, D=D, K=K, vis=vis, ratio=ratio)
+            ri, rl, _, _ = O.topk_rows(one, qb[r0: r0 + L], kk, w[r0: r0 + L], np.arange(L), pool_coef=c)
+            for j in range(L):
+                assert ln[r0 + j] == rl[j], (vis, b, j)
+                assert idx[r0 + j, : ln[r0 + j]].tolist() == (ri[j, : rl[j]] + shift).tolist(), (vis, b, j)
+        full = [stride] * len(lens)
+        a = O.topk_rows_padded(prob, qb, keys_all, w, rows, full, stride, pool_coef=c)
+        bnd = [stride * i for i in range(len(lens) + 1)]
+        d = O.topk_rows_docs(prob, qb, keys_all, w, rows, bnd, pool_coef=c)
+        assert np.array_equal(a[0], d[0]) and np.array_equal(a[1], d[1]), vis
+
+
 def pin_fp8_scales(O):
     """An FP8 value means code * row scale: doubling every key scale doubles
     every score and leaves the selection unchanged; a per-(query, head) scale
@@ -715,6 +757,7 @@ PINS = [
     pin_pair_regions,
     pin_documents,
     pin_documents_compressed,
+    pin_padded_batch,
     pin_fp8_scales,
     pin_witness,
 ]

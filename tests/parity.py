@@ -43,13 +43,27 @@ def host_inputs(inp, rows):
     return h
 
 
-def oracle_rows(wl, inp, rows):
+def oracle_rows(wl, inp, rows, threads=1):
+    """The oracle on the given query rows; with threads > 1 the rows are spread
+    over host threads, one row at a time per thread (NumPy's BLAS held to one
+    thread per call).  Each row is the same plain computation either way."""
     h = host_inputs(inp, rows)
     prob = wl.problem()
     keys = oracle.decode_keys_for(prob, h["k"], h["k_scale"], h["pool_coef"])
-    idx, ln, sc, tau = oracle.topk_rows(prob, h["q_rows"], h["k"], h["w_rows"], rows,
-                                        q_scale_rows=h["q_scale_rows"], k_scale=h["k_scale"],
-                                        pool_coef=h["pool_coef"], keys_f64=keys)
+
+    def run(sl):
+        return oracle.topk_rows(prob, h["q_rows"][sl], h["k"], h["w_rows"][sl], rows[sl],
+                                q_scale_rows=None if h["q_scale_rows"] is None else h["q_scale_rows"][sl],
+                                k_scale=h["k_scale"], pool_coef=h["pool_coef"], keys_f64=keys)
+
+    if threads <= 1:
+        idx, ln, sc, tau = run(slice(None))
+    else:
+        import concurrent.futures as cf
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1), cf.ThreadPoolExecutor(threads) as ex:
+            parts = list(ex.map(run, [slice(i, i + 1) for i in range(len(rows))]))
+        idx, ln, sc, tau = (np.concatenate([p[j] for p in parts]) for j in range(4))
     return dict(idx=idx, len=ln, score=sc, tau=tau, keys=keys, host=h)
 
 
@@ -69,8 +83,10 @@ def assert_exact(gpu, ref, rows):
     assert np.all(both_nan | (gs.astype(np.float64) == rs)), "scores differ"
 
 
-def assert_tolerant(wl, gpu, ref, rows, rel=REL, min_recall=0.9999):
-    """Index-set parity under the tolerance rule; returns the mean recall."""
+def assert_tolerant(wl, gpu, ref, rows, rel=REL, min_recall=0.9999, stats=None):
+    """Index-set parity under the tolerance rule; returns the mean recall
+    (and, given a dict `stats`, fills in the minimum recall and the largest
+    score error relative to max(|s_ref|, |tau|))."""
     gi, gl, gs = (x.cpu().numpy() for x in gpu)
     gi, gl, gs = gi[rows], gl[rows], gs[rows]
     m = wl.ratio if wl.visibility == W.POOLED else 1
@@ -114,6 +130,14 @@ def assert_tolerant(wl, gpu, ref, rows, rel=REL, min_recall=0.9999):
             scale = np.maximum(np.abs(s_ref), abs(tau) if not math.isnan(tau) else np.abs(s_ref).max())
             err = np.abs(sel - s_ref)
             assert np.all(err <= rel * np.maximum(scale, 1e-30)), (t, err.max(), scale.min())
+            if stats is not None:
+                stats["max_rel_score_err"] = max(stats.get("max_rel_score_err", 0.0),
+                                                 float(np.max(err / np.maximum(scale, 1e-30))))
     mean = float(np.mean(recalls)) if recalls else 1.0
+    if stats is not None:
+        stats["mean_recall"] = mean
+        stats["min_recall"] = float(np.min(recalls)) if recalls else 1.0
+        stats["rows"] = len(recalls)
+        stats["rows_with_differences"] = int(sum(r < 1.0 for r in recalls))
     assert mean >= min_recall, mean
     return mean

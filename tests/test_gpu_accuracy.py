@@ -1,0 +1,73 @@
+"""Accuracy of the tensor-core scores against FP64, as a fraction of
+|k| * sum_h |w_h| |q_h| (real values, scales included): the quantity the
+pruning certificate's and the witness threshold's safety margins are stated
+in.  The margins are 2^-11 (certificate, BF16 and FP8) and 2^-12 / 2^-9
+(witness seeds, BF16 / FP8); each must stay at least four times above the
+measured error.  Every visible key is selected (K = T), so out_score carries
+the score of every (query, key) pair.
+
+Inputs: N(0,1) as in the workloads, and |N(0,1)| for q and k, where every
+product of a dot product has the same sign and the partial sums only grow
+(the largest accumulation error relative to the norms)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_weighted_relu_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+CERT_MARGIN = 2.0 ** -11
+WITNESS_MARGIN = {"bf16": 2.0 ** -12, "fp8": 2.0 ** -9}
+
+
+def _inputs(dtype, values, S, T, H, D, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q = torch.randn((S, H, D), generator=g, device="cuda")
+    k = torch.randn((T, D), generator=g, device="cuda")
+    if values == "positive":
+        q, k = q.abs(), k.abs()
+    w = torch.randn((S, H), generator=g, device="cuda") / math.sqrt(H)
+    if dtype == "fp8":
+        qc, qs = W._quantise_e4m3_rows(q)
+        kc, ks = W._quantise_e4m3_rows(k)
+        return dict(q=qc, k=kc, w=w, q_scale=qs, k_scale=ks)
+    return dict(q=q.to(torch.bfloat16), k=k.to(torch.bfloat16), w=w, q_scale=None, k_scale=None)
+
+
+def _decode(dtype, codes, scale):
+    b = W.to_host_bits(codes)
+    if dtype == "fp8":
+        return oracle.decode_e4m3(b) * np.asarray(W.to_host_bits(scale), np.float64)[..., None]
+    return oracle.decode_bf16(b)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("values", ["gauss", "positive"])
+def test_score_error_within_margins(cuda_ok, dtype, values):
+    from head_weighted_relu_b200 import indexer as I
+    S, T, H, D = 256, 2048, 64, 128
+    inp = _inputs(dtype, values, S, T, H, D, seed=81 + (dtype == "fp8") + 2 * (values == "positive"))
+    idx, ln, sc = I.topk(inp["q"], inp["k"], inp["w"], T, q_pos0=T - S, q_scale=inp["q_scale"],
+                         k_scale=inp["k_scale"], with_scores=True)
+    torch.cuda.synchronize()
+    idx, ln, sc = idx.cpu().numpy(), ln.cpu().numpy(), sc.cpu().numpy().astype(np.float64)
+    q = _decode(dtype, inp["q"], inp["q_scale"])           # [S, H, D] real values
+    k = _decode(dtype, inp["k"], inp["k_scale"])           # [T, D]
+    w = W.to_host_bits(inp["w"]).astype(np.float64)       # [S, H]
+    kn = np.linalg.norm(k, axis=1)
+    worst = 0.0
+    for t in range(S):
+        n = T - S + t + 1
+        assert ln[t] == n and np.array_equal(idx[t, :n], np.arange(n))   # every visible key
+        s_ref = oracle.score_keys(q[t], w[t], k[:n])
+        scale = kn[:n] * float(np.abs(w[t]) @ np.linalg.norm(q[t], axis=1))
+        worst = max(worst, float(np.max(np.abs(sc[t, :n] - s_ref) / scale)))
+    print(f"{dtype} {values}: max |s_gpu - s_fp64| / (|k| sum_h |w_h||q_h|) = {worst:.3e} "
+          f"(2^{math.log2(worst) if worst > 0 else float('-inf'):.2f})")
+    assert worst * 4 <= CERT_MARGIN, worst
+    assert worst * 4 <= WITNESS_MARGIN[dtype], worst

@@ -81,3 +81,91 @@ def test_docs_reject_bad_bounds(cuda_ok):
     for bad in ([0, 50, 50, 100], [0, 120], [10, 100], [0]):
         with pytest.raises(I.IndexerError):
             I.indexer_docs_workspace_bytes(prob, bad)
+
+
+# ---------------------------------------------------------------------------
+# Padded batches and the watch lengths in both batch forms
+# ---------------------------------------------------------------------------
+
+WATCH = [3, 4, 5, 7, 8, 9]   # "Module 06 — DSA & KPool", §3 (tests/golden/kpool_watch_lengths.txt)
+
+
+def _run_padded(wl, inp, lens, stride):
+    from head_weighted_relu_b200 import indexer as I
+    prob = I.make_problem(wl.S, wl.T, wl.H, wl.D, wl.K, wl.visibility, wl.ratio, wl.dtype, wl.q_pos0)
+    width = I.indexer_out_width(prob)
+    idx = torch.full((wl.S, width), -7, dtype=torch.int32, device="cuda")
+    ln = torch.full((wl.S,), -7, dtype=torch.int32, device="cuda")
+    sc = torch.full((wl.S, width), -7.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(I.indexer_padded_workspace_bytes(prob, lens, stride), dtype=torch.uint8, device="cuda")
+    I.indexer_topk_padded(prob, inp["q"], inp["k"], inp["w"], inp["q_scale"], inp["k_scale"], inp["pool_coef"],
+                          lens, stride, idx, ln, sc, ws)
+    torch.cuda.synchronize()
+    assert I.indexer_read_status(ws) == 0
+    return idx, ln, sc
+
+
+def _oracle_padded(wl, inp, lens, stride):
+    rows = np.arange(wl.S, dtype=np.int64)
+    h = parity.host_inputs(inp, rows)
+    idx, ln, sc, tau = oracle.topk_rows_padded(wl.problem(), h["q_rows"], h["k"], h["w_rows"], rows, lens, stride,
+                                               q_scale_rows=h["q_scale_rows"], k_scale=h["k_scale"],
+                                               pool_coef=h["pool_coef"])
+    return dict(idx=idx, len=ln, score=sc, tau=tau, host=h)
+
+
+@pytest.mark.parametrize("vis,ratio,K", [(W.TOKEN, 1, 4), (W.COMPRESSED, 4, 4), (W.POOLED, 4, 8)])
+def test_watch_lengths_padded_and_packed(cuda_ok, vis, ratio, K):
+    """The watch lengths as a padded batch (stride 12) and as a packed batch of
+    documents; in the packed form a pool at a document's end would span the
+    boundary if pools were formed on the global grid (documents start at 3, 7,
+    12, 19 and 27).  Integer inputs: bit-exact against the oracle."""
+    stride = 12
+    S = stride * len(WATCH)
+    T = S // ratio if vis == W.COMPRESSED else S
+    wl = W.Workload("watch_pad", S=S, T=T, H=32, D=128, K=K, visibility=vis, ratio=ratio, seed=86 + vis,
+                    values="int")
+    inp = W.generate(wl, "cuda")
+    gpu = _run_padded(wl, inp, WATCH, stride)
+    ref = _oracle_padded(wl, inp, WATCH, stride)
+    parity.assert_exact(gpu, ref, np.arange(S))
+    gl = gpu[1].cpu().numpy()
+    for b, L in enumerate(WATCH):
+        assert (gl[b * stride + L:(b + 1) * stride] == 0).all()   # padding rows select nothing
+    if vis == W.COMPRESSED:
+        return   # packed documents of compressed keys must start on whole keys; the watch lengths do not
+    bounds = np.concatenate([[0], np.cumsum(WATCH)]).tolist()
+    n = bounds[-1]
+    pw = W.Workload("watch_docs", S=n, T=n, H=32, D=128, K=K, visibility=vis, ratio=ratio, seed=96 + vis,
+                    values="int")
+    pin = W.generate(pw, "cuda")
+    parity.assert_exact(_run_docs(pw, pin, bounds), _oracle_docs(pw, pin, bounds), np.arange(n))
+
+
+def test_padded_gaussian_and_split_path(cuda_ok):
+    """Longer padded sequences on Gaussian inputs, one of them empty and one a
+    few rows long; a stride of 9,000 makes the short sequences take the split
+    key-range path."""
+    stride = 9000
+    lens = [9000, 0, 5, 4097]
+    S = stride * len(lens)
+    wl = W.Workload("pad_gauss", S=S, T=S, H=64, D=128, K=256, seed=87)
+    inp = W.generate(wl, "cuda")
+    gpu = _run_padded(wl, inp, lens, stride)
+    rows = np.concatenate([np.arange(0, 600), np.arange(8990, 9010), np.arange(18000, 18010),
+                           np.arange(27000, 27000 + 4100)])
+    h = parity.host_inputs(inp, rows)
+    idx, ln, sc, tau = oracle.topk_rows_padded(wl.problem(), h["q_rows"], h["k"], h["w_rows"], rows, lens, stride)
+    ref = dict(idx=idx, len=ln, score=sc, tau=tau, host=h,
+               keys=oracle.decode_keys_for(wl.problem(), h["k"]))
+    parity.assert_tolerant(wl, gpu, ref, rows)
+
+
+def test_padded_rejects_bad_shapes(cuda_ok):
+    from head_weighted_relu_b200 import indexer as I
+    ok = I.make_problem(24, 24, 64, 128, 8)
+    assert I.indexer_padded_workspace_bytes(ok, [12, 5], 12) >= 256
+    for prob, lens, stride in ((ok, [13, 5], 12), (ok, [12, 5], 11), (I.make_problem(24, 24, 64, 128, 8, q_pos0=0), [12], 12),
+                               (I.make_problem(24, 5, 64, 128, 8, I.COMPRESSED, 4), [12, 12], 12)):
+        with pytest.raises(I.IndexerError):
+            I.indexer_padded_workspace_bytes(prob, lens, stride)

@@ -48,6 +48,10 @@ MUTATIONS = {
                                        "vis = j[(j > b // ratio) & (ratio * j + ratio - 1 <= g)]"),
     "compressed_doc_start_ignored": ("vis = j[(j >= b // ratio) & (ratio * j + ratio - 1 <= g)]",
                                      "vis = j[(ratio * j + ratio - 1 <= g)]"),
+    "padding_rows_select": ("            continue                                  # a padding query row",
+                            "            pass"),
+    "padded_pools_on_global_grid": ("            pos = (start + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)",
+                                    "            pos = (start // 8 * 8 + sel[:, None] * ratio + np.arange(ratio)[None, :]).reshape(-1)"),
     "witness_kth_off_by_one": ("taus[r] = float(np.sort(s)[::-1][ksel - 1])", "taus[r] = float(np.sort(s)[::-1][ksel - 2])"),
 }
 

@@ -51,6 +51,7 @@ def test_noalloc_matches_workspace_entry_point(cuda_ok, wl):
         same = torch.isnan(sc) & torch.isnan(ref_sc)
         close = (sc - ref_sc).abs() <= parity.REL * ref_sc.abs().clamp_min(1e-30)
         assert bool((same | close).all())
+        assert I.indexer_noalloc_read_status() == 0   # no wait timed out, no buffer overflowed
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_ok):
