@@ -270,7 +270,7 @@ def cpu_baseline(wl, inp, all_s=12.0, one_s=6.0):
                 one_core_value=v_one,
                 extrapolated_full_problem_s={"all_cores": total / (v_all * 1e9), "one_core": total / (v_one * 1e9),
                                              "note": "extrapolation: the problem's pairs / the sampled rate"},
-                sample=(f"{wl.name}: the first {n_all} of the 1,024 seeded parity rows on {r.cores} threads "
+                sample=(f"{wl.name}: {n_all} of the 1,024 seeded parity rows on {r.cores} threads "
                         f"({p_all} pairs, {t_all:.1f} s), the first {n_one} on one thread ({p_one} pairs, "
                         f"{t_one:.1f} s); NumPy FP64, full score row + stable sort per row, one row per thread"))
 
@@ -302,9 +302,9 @@ def run_reference(args, wl, world, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(wl, world, args.scaling),
         "cpu_baseline": {"value": val, "unit": "Gpairs/s", "cores": r.cores, "kind": "oracle",
-                         "sample": f"{rows_done} of the 1,024 seeded parity rows of {wl.name} "
-                                   f"({pairs_done} pairs, {secs:.1f} s over {args.steps} steps), "
-                                   "one row per thread on every core"},
+                         "sample": f"{rows_done} rows taken in turn from the 1,024 seeded parity rows of "
+                                   f"{wl.name} ({pairs_done} pairs, {secs:.1f} s over {args.steps} steps of "
+                                   "at most 3 s or one pass), one row per thread on every core"},
         "e2e": {"value": val, "unit": "Gpairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 

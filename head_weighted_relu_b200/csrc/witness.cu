@@ -14,9 +14,10 @@
 //   eps * |k| * sum_h |w_h| |q_h|   (times the key scale for FP8).
 // Each dot product over D = 128 exact products carries at most about
 // D * 2^-24 = 2^-17 of |q_h| |k| in FP32 on either side, the head sums far
-// less; eps = 2^-12 for BF16 leaves a wide factor over that.  FP8 takes
-// eps = 2^-9, four times the pruning certificate's margin, since the
-// precision of the FP8 tensor-core accumulation is not documented.  The
+// less.  The tensor-core scores, measured against FP64 on inputs whose
+// products all have one sign (the largest accumulation error relative to the
+// norms), stay within 2^-23 of |k| sum_h |w_h| |q_h| for BF16 and for FP8
+// (kind::f8f6f4) alike, so eps = 2^-12 leaves a wide factor for both.  The
 // threshold is the K-th largest lowered score over the row's distinct visible
 // seeds, so at least K keys score at or above it in the scoring kernel and
 // the exact top-K is unchanged.  A margin that fell short could only put the
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kSeedThreads) witness_scores_kernel(const Witn
           }
           s = fmaf(ws[h], fmaxf((x0 + x1) + (x2 + x3), 0.f), s);
         }
-        float margin = (wp.fp8 ? 0x1p-9f : 0x1p-12f) * (sqrtf(kn2) * (1.0f + 0x1p-18f)) * amp;
+        float margin = 0x1p-12f * (sqrtf(kn2) * (1.0f + 0x1p-18f)) * amp;
         if (wp.fp8) {
           const float ks = wp.k_scale[r];
           s *= ks;

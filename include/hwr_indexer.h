@@ -234,7 +234,7 @@ indexer_status indexer_topk_host(const indexer_problem* p, const void* q, const 
  *          ascending order are used whole, and no key counts twice).
  * Each row's remaining seeds are scored exactly in FP32 on CUDA cores,
  * lowered by a margin that covers the difference to the tensor-core scores
- * (eps |k| sum_h |w_h||q_h| with eps = 2^-12 for BF16 and 2^-9 for FP8, times
+ * (eps |k| sum_h |w_h||q_h| with eps = 2^-12 for BF16 and FP8, times
  * the key scale for FP8), and their K-th
  * largest (K/ratio-th for POOLED) becomes the query's starting threshold; with
  * fewer seeds than that the query starts from no threshold.  Keys below the

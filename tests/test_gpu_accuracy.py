@@ -1,9 +1,9 @@
 """Accuracy of the tensor-core scores against FP64, as a fraction of
 |k| * sum_h |w_h| |q_h| (real values, scales included): the quantity the
 pruning certificate's and the witness threshold's safety margins are stated
-in.  The margins are 2^-11 (certificate, BF16 and FP8) and 2^-12 / 2^-9
-(witness seeds, BF16 / FP8); each must stay at least four times above the
-measured error.  Every visible key is selected (K = T), so out_score carries
+in.  The margins are 2^-11 (certificate) and 2^-12 (witness seeds), for BF16
+and FP8 alike; each must stay at least four times above the measured error
+(measured on B200: about 2^-23.3 at worst, for both types).  Every visible key is selected (K = T), so out_score carries
 the score of every (query, key) pair.
 
 Inputs: N(0,1) as in the workloads, and |N(0,1)| for q and k, where every
@@ -22,7 +22,7 @@ from head_weighted_relu_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 CERT_MARGIN = 2.0 ** -11
-WITNESS_MARGIN = {"bf16": 2.0 ** -12, "fp8": 2.0 ** -9}
+WITNESS_MARGIN = {"bf16": 2.0 ** -12, "fp8": 2.0 ** -12}
 
 
 def _inputs(dtype, values, S, T, H, D, seed):
