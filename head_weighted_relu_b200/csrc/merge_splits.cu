@@ -312,7 +312,16 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
       rb_load(rb, buf, n, etid);
       RegCut c{0u, 0xFFFFFFFFu, false, n};
       if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(mp.ksel), false, 0, hist, st.red, etid, bar_id);
-      kept = rb_compact(rb, n, c, all, st.scan, etid, bar_id, emit);
+      // hist is scratch from here on: pooled entries expand through it
+      kept = rb_compact_steps(rb, n, c, all, st.scan, etid, bar_id,
+                              [&](bool keep, int pos, uint32_t k, uint32_t ix, int first, int count) {
+                                if (m == 1) {
+                                  if (keep) emit(pos, k, ix);
+                                } else {
+                                  emit_expanded(keep, pos, k, ix, first, count, m, orow, srow,
+                                                hist + (etid >> 5) * 64, lane);
+                                }
+                              });
     } else {
       Cut cut{0u, 0xFFFFFFFFu};
       if (!all) cut = m_topk_cut(buf, n, static_cast<uint32_t>(mp.ksel), hist, st.red, etid, bar_id);

@@ -388,30 +388,37 @@ __device__ int wg_compact(const uint2* buf, int n, Cut c, bool keep_all, int32_t
 
 // ------------------------------------------------------------------------
 // Register-resident selection: the warpgroup holds the whole candidate
-// buffer in registers, thread etid holding the contiguous entries
-// [32*etid, 32*etid + 32), so every pass over it runs without memory round
-// trips and order-preserving compaction needs one prefix scan.  Used whenever
-// the buffer fits (capacity <= 4,096 entries, i.e. budgets up to 2,048).
+// buffer in registers.  Entry e lives in warp e / 1024, register
+// (e % 1024) / 32, lane e % 32, so each register step of a warp covers 32
+// consecutive entries: loading the buffer and writing kept entries back (or
+// out) are coalesced 256-byte accesses, and order-preserving compaction needs
+// one ballot per step and one exchange of per-warp counts.  Used whenever the
+// buffer fits (capacity <= 4,096 entries, i.e. budgets up to 2,048).
 // ------------------------------------------------------------------------
 constexpr int kRegEntries = 32;
 constexpr int kRegCap = kRegEntries * kBM;
+constexpr int kWarpEntries = kRegEntries * 32;   // entries held by one warp
 
 struct RegBuf {
   uint32_t key[kRegEntries];
   uint32_t idx[kRegEntries];
 };
 
+// Register r of this thread holds buffer position (etid / 32) * 1024 +
+// 32 r + etid % 32; it is valid iff 32 r < rb_room(n, etid).
+__device__ __forceinline__ int rb_room(int n, int etid) {
+  return n - (etid >> 5) * kWarpEntries - (etid & 31);
+}
+
 __device__ __forceinline__ void rb_load(RegBuf& b, const uint2* buf, int n, int etid) {
-  const int base = etid * kRegEntries;
-  const uint4* v = reinterpret_cast<const uint4*>(buf + base);
+  const int room = rb_room(n, etid);
+  const uint2* src = buf + (etid >> 5) * kWarpEntries + (etid & 31);
 #pragma unroll
-  for (int r = 0; r < kRegEntries; r += 2) {
-    uint4 e = make_uint4(0u, 0u, 0u, 0u);
-    if (base + r < n) e = v[r >> 1];  // n entries are valid; the pair's tail is masked below
-    b.key[r] = e.x;
-    b.idx[r] = e.y;
-    b.key[r + 1] = e.z;
-    b.idx[r + 1] = e.w;
+  for (int r = 0; r < kRegEntries; ++r) {
+    uint2 v = make_uint2(0u, 0u);
+    if (32 * r < room) v = src[32 * r];
+    b.key[r] = v.x;
+    b.idx[r] = v.y;
   }
 }
 
@@ -426,16 +433,16 @@ __device__ __forceinline__ uint32_t rb_field(const RegBuf& b, int r, bool idx_fi
 __device__ inline void rb_maxmin(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t& mx,
                           uint32_t& mn, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
-  const int base = etid * kRegEntries;
   mx = 0u;
   mn = 0xFFFFFFFFu;
+  const int room = rb_room(n, etid);
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r) {
-    if (base + r < n && (!filt || b.key[r] == fval)) {
-      const uint32_t f = rb_field(b, r, idx_field);
-      mx = max(mx, f);
-      mn = min(mn, f);
-    }
+    // branch-free: every condition is a predicate, every update a select
+    const bool ok = (32 * r < room) & (!filt | (b.key[r] == fval));
+    const uint32_t f = rb_field(b, r, idx_field);
+    mx = max(mx, ok ? f : 0u);
+    mn = min(mn, ok ? f : 0xFFFFFFFFu);
   }
   mx = warp_max_u32(mx);
   mn = warp_min_u32(mn);
@@ -454,63 +461,66 @@ struct Digit {
   uint32_t cnt;    // entries in digit d
 };
 
-// One MSB-first radix pass over bits [lo - width, lo) of the valid entries
-// whose bits [lo, 32) equal prefix's.  Bin b of the histogram sits at word
-// ((b % per) << 7) + b / per, so the 128 owner threads, each summing `per`
-// consecutive bins, read distinct banks.
-__device__ inline Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t prefix, int lo,
-                         int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
+// One radix pass over the valid entries whose ranked value f lies in
+// [base, base + 2^(shift + width)): digit (f - base) >> shift, 2^width bins,
+// counted from the top.  Digits are offsets from a base rather than bit
+// fields of f, so a range of values that straddles a power of two (where all
+// exponent bits of the ordered score change) still spreads over the bins.
+// hist[0, 2^width) must be zero on entry and is zero again on return.  Every
+// thread adds its entries to the histogram; warp 0 then finds the digit:
+// lane L sums bins [L*per, L*per+per) (rotated so that the lanes read
+// distinct banks), a suffix scan over the lanes finds the lane holding the
+// rank-th largest, a second scan over that lane's bins finds the digit, and
+// the warp clears the bins.  Two barriers.
+__device__ inline Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t base,
+                         int shift, int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
-  const int base = etid * kRegEntries;
-  const int shift = lo - width;
   const int nb = 1 << width;
-  const int lper = width > 7 ? width - 7 : 0;
-  const int per = 1 << lper;
-  for (int i = etid; i < nb; i += kBM) hist[i] = 0u;
-  named_bar(bar_id, kBM);
+  const unsigned long long span = 1ull << (shift + width);
+  const int room = rb_room(n, etid);
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r) {
-    if (base + r < n && (!filt || b.key[r] == fval)) {
-      const uint32_t f = rb_field(b, r, idx_field);
-      if (lo >= 32 || (f >> lo) == (prefix >> lo)) {
-        const uint32_t bin = (f >> shift) & static_cast<uint32_t>(nb - 1);
-        atomicAdd(&hist[((bin & static_cast<uint32_t>(per - 1)) << 7) + (bin >> lper)], 1u);
-      }
-    }
+    const uint32_t f = rb_field(b, r, idx_field);
+    // branch-free: every condition is a predicate
+    const bool ok = (32 * r < room) & (!filt | (b.key[r] == fval)) & (f >= base) &
+                    (static_cast<unsigned long long>(f - base) < span);
+    if (ok) atomicAdd(&hist[(f - base) >> shift], 1u);
   }
   named_bar(bar_id, kBM);
-  const bool owner = etid < (nb >> lper);
-  uint32_t local = 0u;
-  if (owner)
-    for (int k = 0; k < per; ++k) local += hist[(k << 7) + etid];
-  uint32_t incl = local;  // sum over lanes >= this lane
+  if (wq == 0) {
+    const int per = nb >= 32 ? nb >> 5 : 1;   // bins per lane (a power of two)
+    const int owners = nb >= 32 ? 32 : nb;
+    uint32_t local = 0u;
+    if (lane < owners)
+      for (int k = 0; k < per; ++k) local += hist[lane * per + ((k + lane) & (per - 1))];
+    uint32_t incl = local;  // entries in bins of lanes >= this lane
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_down_sync(kFullMask, incl, o);
-    if (lane + o < 32) incl += t;
-  }
-  if (lane == 0) red[wq] = incl;
-  named_bar(bar_id, kBM);
-  uint32_t higher = 0u;
-  for (int w2 = wq + 1; w2 < 4; ++w2) higher += red[w2];
-  const uint32_t excl = incl - local + higher;  // entries in bins owned by higher threads
-  if (owner && local > 0u && excl < rank && rank <= excl + local) {
-    uint32_t acc = excl;
-    for (int k = per - 1; k >= 0; --k) {
-      const uint32_t h = hist[(k << 7) + etid];
-      if (acc + h >= rank) {
-        red[8] = static_cast<uint32_t>(etid * per + k);
-        red[9] = acc;
-        red[10] = h;
-        break;
-      }
-      acc += h;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(kFullMask, incl, o);
+      if (lane + o < 32) incl += t;
     }
+    const uint32_t excl = incl - local;
+    const int ls = max(__ffs(__ballot_sync(kFullMask, lane < owners && excl < rank && rank <= incl)) - 1, 0);
+    const uint32_t above = __shfl_sync(kFullMask, excl, ls);
+    // inside lane ls's bins: lane j takes bin ls * per + j
+    const uint32_t h = lane < per ? hist[ls * per + lane] : 0u;
+    uint32_t inc2 = h;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(kFullMask, inc2, o);
+      if (lane + o < 32) inc2 += t;
+    }
+    const uint32_t ex2 = inc2 - h;
+    if (lane < per && above + ex2 < rank && rank <= above + inc2) {
+      red[8] = static_cast<uint32_t>(ls * per + lane);
+      red[9] = above + ex2;
+      red[10] = h;
+    }
+    __syncwarp();
+    for (int i = lane; i < nb; i += 32) hist[i] = 0u;
   }
   named_bar(bar_id, kBM);
-  const Digit out{red[8], red[9], red[10]};
-  named_bar(bar_id, kBM);
-  return out;
+  return Digit{red[8], red[9], red[10]};
 }
 
 // A cut of a buffer to its top `ksel`: keep key >= v when `ge`, otherwise keep
@@ -522,80 +532,160 @@ struct RegCut {
   int kept;
 };
 
-// MSB-first radix select of the ksel-th largest (ordered score, then lowest
-// index), starting below the bits every entry shares.  With `approx`, stops
-// after the first pass if keeping the whole digit that holds the ksel-th entry
+// Entries at most this many in the bin that holds the ksel-th largest are
+// sorted in one warp instead of further radix passes.
+constexpr int kSmallSel = 64;
+
+// Sorts 64 keys held as v[j] = element 32 j + lane into descending order
+// (bitonic network; pairs at distance 32 sit in the same lane).
+__device__ __forceinline__ void warp_sort64_desc(unsigned long long (&v)[2], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int s = k >> 1; s > 0; s >>= 1) {
+      unsigned long long nv[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int i = j * 32 + lane;
+        const unsigned long long other = s == 32 ? v[j ^ 1] : __shfl_xor_sync(kFullMask, v[j], s);
+        // in a block sorted descending the lower index of a pair takes the larger
+        const bool take_max = ((i & s) == 0) == ((i & k) == 0);
+        nv[j] = take_max ? (v[j] > other ? v[j] : other) : (v[j] < other ? v[j] : other);
+      }
+      v[0] = nv[0];
+      v[1] = nv[1];
+    }
+  }
+}
+
+// The cut when the remaining candidates -- the entries whose ordered score
+// lies in [base, base + 2^shift) -- number at most kSmallSel: they are
+// gathered into shared memory (hist[512, 640), free after the passes), warp
+// 0 sorts them by (ordered score desc, index asc) and the rank-th of them
+// gives v and the index cut.  red[12] counts the gathered entries (cleared by
+// the caller before its first barrier).
+__device__ inline RegCut rb_small_select(const RegBuf& b, int n, uint32_t base, int shift, uint32_t rank,
+                                         uint32_t ksel, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
+  const int lane = etid & 31, wq = etid >> 5;
+  const int room = rb_room(n, etid);
+  const unsigned long long span = 1ull << shift;
+  uint2* list = reinterpret_cast<uint2*>(hist + 512);
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r) {
+    const uint32_t k = b.key[r];
+    const bool in = (32 * r < room) & (k >= base) & (static_cast<unsigned long long>(k - base) < span);
+    if (in) list[atomicAdd(&red[12], 1u)] = make_uint2(k, b.idx[r]);
+  }
+  named_bar(bar_id, kBM);
+  if (wq == 0) {
+    const uint32_t m = red[12];
+    unsigned long long v[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t i = j * 32 + lane;
+      // (score, ~index): larger is better; unused slots sort last
+      v[j] = i < m ? (static_cast<unsigned long long>(list[i].x) << 32) | (~list[i].y) : 0ull;
+    }
+    warp_sort64_desc(v, lane);
+    const uint32_t at = rank - 1;  // 0-based position of the rank-th best
+    const unsigned long long w = __shfl_sync(kFullMask, at < 32 ? v[0] : v[1], at & 31);
+    if (lane == 0) {
+      red[8] = static_cast<uint32_t>(w >> 32);
+      red[9] = ~static_cast<uint32_t>(w);
+    }
+  }
+  named_bar(bar_id, kBM);
+  return {red[8], red[9], false, static_cast<int>(ksel)};
+}
+
+// Radix select of the ksel-th largest (ordered score, then lowest index).
+// Passes of up to 10 bits walk down from the span [min, max] of the scores:
+// each pass narrows the range holding the ksel-th entry to one bin.  With
+// `approx`, stops after the first pass if keeping everything from that bin up
 // keeps at most `room` entries: a safe lower bound for a running threshold.
+// Once the bin holding the ksel-th entry has at most kSmallSel entries, they
+// are sorted in one warp (rb_small_select) instead of further passes.
 __device__ inline RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int room, uint32_t* hist,
                          uint32_t* red, int etid, int bar_id) {
   uint32_t mx, mn;
+  // the passes keep the histogram zero between them; the barrier of the
+  // max / min below orders this clearing (and of the gather counter) before
+  // the first pass
+  for (int i = etid; i < kHistBins; i += kBM) hist[i] = 0u;
+  if (etid == 0) red[12] = 0u;
   rb_maxmin(b, n, false, false, 0u, mx, mn, red, etid, bar_id);
-  uint32_t prefix = mx, above = 0u, cnt = static_cast<uint32_t>(n), rank = ksel;
+  uint32_t base = mn, above = 0u, cnt = static_cast<uint32_t>(n), rank = ksel;
   if (mx != mn) {
-    int lo = 32 - __clz(mx ^ mn);
-    prefix = lo >= 32 ? 0u : (mx >> lo) << lo;
+    int shift = 32 - __clz(mx - mn);  // bits of the span of the scores
     bool first = true;
-    while (lo > 0) {
-      const int width = lo < kDigitBits ? lo : kDigitBits;
-      const Digit dg = rb_pass(b, n, false, false, 0u, prefix, lo, width, rank, hist, red, etid, bar_id);
-      lo -= width;
-      prefix |= dg.d << lo;
+    while (shift > 0) {
+      const int width = shift < kDigitBits ? shift : kDigitBits;
+      shift -= width;
+      const Digit dg = rb_pass(b, n, false, false, 0u, base, shift, width, rank, hist, red, etid, bar_id);
+      base += dg.d << shift;
       above += dg.above;
       rank -= dg.above;
       cnt = dg.cnt;
       if (approx && first && static_cast<int>(above + cnt) <= room)
-        return {prefix, 0u, true, static_cast<int>(above + cnt)};
+        return {base, 0u, true, static_cast<int>(above + cnt)};
       first = false;
+      if (cnt <= static_cast<uint32_t>(kSmallSel))
+        return rb_small_select(b, n, base, shift, rank, ksel, hist, red, etid, bar_id);
     }
   }
-  // prefix is now v, the ksel-th largest ordered score; `rank` of the `cnt`
+  // base is now v, the ksel-th largest ordered score; `rank` of the `cnt`
   // entries tied at v make the cut
-  if (rank >= cnt) return {prefix, 0xFFFFFFFFu, false, static_cast<int>(above + cnt)};
+  if (rank >= cnt) return {base, 0xFFFFFFFFu, false, static_cast<int>(above + cnt)};
+  if (cnt <= static_cast<uint32_t>(kSmallSel))
+    return rb_small_select(b, n, base, 0, rank, ksel, hist, red, etid, bar_id);
+  // many ties at v: the rank-th largest ~index among them, by the same passes
+  const uint32_t v = base;
   uint32_t imx, imn;
-  rb_maxmin(b, n, true, true, prefix, imx, imn, red, etid, bar_id);
-  uint32_t ip = imx;
+  rb_maxmin(b, n, true, true, v, imx, imn, red, etid, bar_id);
+  uint32_t ibase = imn;
   if (imx != imn) {
-    int lo = 32 - __clz(imx ^ imn);
-    ip = lo >= 32 ? 0u : (imx >> lo) << lo;
-    uint32_t irank = rank;
-    while (lo > 0) {
-      const int width = lo < kDigitBits ? lo : kDigitBits;
-      const Digit dg = rb_pass(b, n, true, true, prefix, ip, lo, width, irank, hist, red, etid, bar_id);
-      lo -= width;
-      ip |= dg.d << lo;
-      irank -= dg.above;
+    int shift = 32 - __clz(imx - imn);
+    while (shift > 0) {
+      const int width = shift < kDigitBits ? shift : kDigitBits;
+      shift -= width;
+      const Digit dg = rb_pass(b, n, true, true, v, ibase, shift, width, rank, hist, red, etid, bar_id);
+      ibase += dg.d << shift;
+      rank -= dg.above;
     }
   }
-  return {prefix, ~ip, false, static_cast<int>(ksel)};
+  return {v, ~ibase, false, static_cast<int>(ksel)};
 }
 
-// Calls emit(pos, key, idx) for every kept entry, pos counting kept entries in
-// buffer (key) order; returns the number kept.  Each thread counts its kept
-// entries, one scan over the warpgroup gives its first position.  All reads
-// are from registers, so emitting back into the same buffer is safe.
-template <class Emit>
-__device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all, int32_t* red_i, int etid,
-                          int bar_id, Emit emit) {
+// Order-preserving compaction of the register buffer; returns the number
+// kept.  Each warp counts its kept entries (one ballot per register step),
+// the counts are exchanged once, and a second ballot pass gives every kept
+// entry its position pos (counting kept entries in buffer, i.e. key, order).
+// The kept entries of one warp step land on consecutive positions
+// [first, first + count), so writes are coalesced.  step(keep, pos, key,
+// idx, first, count) is called by every lane of the warp for every register
+// step (keep: this lane's entry is kept), so it may use warp-collective
+// operations.  All reads are from registers: writing back into the same
+// buffer is safe.
+template <class Step>
+__device__ int rb_compact_steps(const RegBuf& b, int n, const RegCut& c, bool keep_all, int32_t* red_i, int etid,
+                                int bar_id, Step step) {
   const int lane = etid & 31, wq = etid >> 5;
-  const int base = etid * kRegEntries;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int room = rb_room(n, etid);
+  // keep: key > v, or key == v and index <= icut (a `ge` cut keeps every
+  // index at v), as one branch-free predicate
+  const uint32_t icut = (keep_all || c.ge) ? 0xFFFFFFFFu : c.icut;
+  const uint32_t v = keep_all ? 0u : c.v;
   auto keep_of = [&](int r) -> bool {
-    if (base + r >= n) return false;
-    if (keep_all) return true;
     const uint32_t k = b.key[r];
-    return c.ge ? (k >= c.v) : (k > c.v || (k == c.v && b.idx[r] <= c.icut));
+    return (32 * r < room) & ((k > v) | ((k == v) & (b.idx[r] <= icut)));
   };
-  int mine = 0;
+  int mine = 0;  // kept entries of this warp
 #pragma unroll
-  for (int r = 0; r < kRegEntries; ++r) mine += keep_of(r) ? 1 : 0;
-  int incl = mine;  // inclusive prefix over lanes <= this lane
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(kFullMask, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) red_i[wq] = incl;
+  for (int r = 0; r < kRegEntries; ++r) mine += __popc(__ballot_sync(kFullMask, keep_of(r)));
+  if (lane == 0) red_i[wq] = mine;
   named_bar(bar_id, kBM);
-  int pos = incl - mine, total = 0;
+  int pos = 0, total = 0;
 #pragma unroll
   for (int w2 = 0; w2 < 4; ++w2) {
     const int t = red_i[w2];
@@ -603,10 +693,45 @@ __device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all
     pos += (w2 < wq) ? t : 0;
   }
 #pragma unroll
-  for (int r = 0; r < kRegEntries; ++r)
-    if (keep_of(r)) emit(pos++, b.key[r], b.idx[r]);
+  for (int r = 0; r < kRegEntries; ++r) {
+    const bool k = keep_of(r);
+    const uint32_t bal = __ballot_sync(kFullMask, k);
+    if (bal != 0u) step(k, pos + __popc(bal & lt), b.key[r], b.idx[r], pos, __popc(bal));
+    pos += __popc(bal);
+  }
   named_bar(bar_id, kBM);
   return total;
+}
+
+// rb_compact_steps with emit(pos, key, idx) called for each kept entry.
+template <class Emit>
+__device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all, int32_t* red_i, int etid,
+                          int bar_id, Emit emit) {
+  return rb_compact_steps(b, n, c, keep_all, red_i, etid, bar_id,
+                          [&](bool keep, int pos, uint32_t k, uint32_t ix, int, int) {
+                            if (keep) emit(pos, k, ix);
+                          });
+}
+
+// One compaction step's kept pools, each expanded to its m token positions
+// ("Module 06 — DSA & KPool", §2), written with consecutive lanes on
+// consecutive output slots: the step's pools go to slots [first * m,
+// (first + count) * m).  Called by every lane of the warp; `stage` is 64
+// words of this warp's shared-memory scratch.  srow (optional) gets each
+// pool's score for each of its tokens.
+__device__ __forceinline__ void emit_expanded(bool keep, int pos, uint32_t key, uint32_t ix, int first, int count,
+                                              int m, int32_t* orow, float* srow, uint32_t* stage, int lane) {
+  if (keep) {
+    stage[pos - first] = ix;
+    stage[32 + pos - first] = key;
+  }
+  __syncwarp();
+  for (int j = lane; j < count * m; j += 32) {
+    const int e = j / m;
+    orow[first * m + j] = static_cast<int32_t>(stage[e]) * m + (j - e * m);
+    if (srow) srow[first * m + j] = key_to_float(stage[32 + e]);
+  }
+  __syncwarp();
 }
 
 // ------------------------------------------------------------------------
@@ -1078,6 +1203,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             };
+            // the same, by warp steps: pooled entries expand with coalesced writes
+            auto step = [&](bool keep, int pos, uint32_t k, uint32_t ix, int first, int count) {
+              if (SPLIT || m == 1) {
+                if (keep) emit(pos, k, ix);
+              } else {
+                emit_expanded(keep, pos, k, ix, first, count, m, orow, srow, hist + (etid >> 5) * 64, etid & 31);
+              }
+            };
             int kept;
             [[maybe_unused]] uint32_t kth = 0u;  // ordered score of the K-th entry kept (0: fewer than K)
             [[maybe_unused]] uint32_t rth = 0u;  // split ranges: ordered score of the r-th entry (0: fewer)
@@ -1086,7 +1219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               rb_load(rb, buf, n, etid);
               RegCut c{0u, 0xFFFFFFFFu, false, n};
               if (!all) c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
-              kept = rb_compact(rb, n, c, all, st->scan, etid, bar_id, emit);
+              // hist is scratch from here on (rb_cut clears it before use)
+              kept = rb_compact_steps(rb, n, c, all, st->scan, etid, bar_id, step);
               if constexpr (SPLIT) {
                 kth = all ? 0u : c.v;
                 // the r-th largest score of the range, r = ceil(K / splits)
