@@ -1018,9 +1018,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           nvis_r[qi] = st->nvis[qi];
         }
         bool any_full = false;
+        // per-key values of the next tile (FP8 key scale, pruning key norm),
+        // loaded one tile ahead so that their latency hides behind the wait
+        // for the accumulator and the head sums
+        float ks_next = 1.f, kn_next = 0.f;
+        {
+          const int32_t key = j * kBM + etid;
+          if constexpr (FP8) ks_next = (j < nt && key < p.n_keys) ? p.k_scale[key] : 0.f;
+          if constexpr (PRUNE) kn_next = (j < nt && key < p.n_keys) ? p.knorm[key] : 0.f;
+        }
         for (; j < nt; ++j) {
           const int a = static_cast<int>(tcount & 1u);
           ++tcount;
+          const int32_t key = j * kBM + etid;
+          const float ks = ks_next, kn = kn_next;
+          if (FP8 || PRUNE) {
+            const int32_t key1 = key + kBM;
+            const bool more = j + 1 < nt && key1 < p.n_keys;
+            if constexpr (FP8) ks_next = more ? p.k_scale[key1] : 0.f;
+            if constexpr (PRUNE) kn_next = more ? p.knorm[key1] : 0.f;
+          }
           // every lane polls (no divergent branch around the wait); the phase
           // is complete for all once any lane has seen it complete
           bool ok = mbar_wait(&bars->accfull[a], (af_bits >> a) & 1u, abort_flag, kWaitLimitNs);
@@ -1029,10 +1046,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           float s[NQW];
 #pragma unroll
           for (int qi = 0; qi < NQW; ++qi) s[qi] = 0.f;
-          const int32_t key = j * kBM + etid;
-          float ks = 1.f, kn = 0.f;
-          if constexpr (FP8) ks = key < p.n_keys ? p.k_scale[key] : 0.f;
-          if constexpr (PRUNE) kn = key < p.n_keys ? p.knorm[key] : 0.f;
           if (ok) {
             tc_fence_after();
             const uint32_t tb = tbase + static_cast<uint32_t>(a * BN);
