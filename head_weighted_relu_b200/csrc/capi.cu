@@ -333,6 +333,7 @@ indexer_status run_topk(const indexer_problem* p, const void* q, const void* k, 
   sp.ranged = pl.ranged;
   sp.ratio = pl.ranged ? p->ratio : 1;
   sp.out_ratio = pl.out_ratio;
+  sp.out_ratio_inv = pl.out_ratio > 1 ? 0xFFFFFFFFu / static_cast<uint32_t>(pl.out_ratio) + 1u : 0u;
   sp.ksel = pl.ksel;
   sp.width = pl.width;
   sp.n_blocks = pl.n_blocks;

@@ -24,6 +24,7 @@ struct ScoreParams {
   int32_t ranged;     // 0: key i visible iff i <= g; 1: key j visible iff ratio*j + ratio - 1 <= g
   int32_t ratio;      // key span for ranged visibility
   int32_t out_ratio;  // 1, or the pool width: each selected pool expands to out_ratio positions + tail
+  uint32_t out_ratio_inv;  // ceil(2^32 / out_ratio) when out_ratio > 1 (division-free pool expansion)
   int32_t ksel;       // keys (pools) to select per query
   int32_t width;      // row stride of out_idx / out_score
   int32_t n_blocks;   // query blocks

@@ -299,6 +299,7 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
     int32_t* orow = mp.out_idx + t * mp.width;
     float* srow = mp.out_score ? mp.out_score + t * mp.width : nullptr;
     const int m = mp.out_ratio;
+    const uint32_t minv = m > 1 ? 0xFFFFFFFFu / static_cast<uint32_t>(m) + 1u : 0u;
     auto emit = [&](int pos, uint32_t k, uint32_t ix) {
       const float sc = key_to_float(k);
       for (int rr = 0; rr < m; ++rr) {
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(kBM) merge_splits_kernel(const MergeParams mp)
                                 if (m == 1) {
                                   if (keep) emit(pos, k, ix);
                                 } else {
-                                  emit_expanded(keep, pos, k, ix, first, count, m, orow, srow,
+                                  emit_expanded(keep, pos, k, ix, first, count, m, minv, orow, srow,
                                                 hist + (etid >> 5) * 64, lane);
                                 }
                               });

@@ -89,6 +89,20 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool v) {
   return r != 0;
 }
 
+// Named barrier that also counts the participating threads whose predicate
+// is true.
+__device__ __forceinline__ uint32_t named_bar_popc(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.popc.u32 %0, %2, %3, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r;
+}
+
 // ----------------------------------------------------------------------- TMA --
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");

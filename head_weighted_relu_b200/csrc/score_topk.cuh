@@ -42,6 +42,8 @@
 // or rejected exactly as a full sort of the score row would.
 #pragma once
 
+#include <cstddef>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -70,8 +72,12 @@ struct WgState {
   uint32_t red[16];      // reduction scratch
   int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
   int32_t scan[4];       // per-warp totals of a register-resident compaction
-  float pq[NQ][kPruneR + 4];  // pruning: folded weights of the kept heads, then Ceff
+  // pruning: folded weights of the kept heads, then Ceff (read as float4)
+  alignas(16) float pq[NQ][kPruneR + 4];
 };
+static_assert(offsetof(WgState<1>, pq) % 16 == 0 && offsetof(WgState<2>, pq) % 16 == 0 &&
+                  offsetof(WgState<8>, pq) % 16 == 0 && sizeof(WgState<1>) % 16 == 0,
+              "pruning weights are read as float4");
 
 template <int STAGES>
 struct Barriers {
@@ -84,6 +90,8 @@ struct Barriers {
   uint32_t tmem_slot;
   int abort;
   int tmem_busy;       // MMAs may still write TMEM: leave it allocated
+  int cut_round;       // raised by a group whose buffer filled: others cut too
+  int seen[4];         // the cut round each epilogue group has taken part in
 };
 
 template <int H, int D, bool FP8>
@@ -718,16 +726,18 @@ __device__ int rb_compact(const RegBuf& b, int n, const RegCut& c, bool keep_all
 // consecutive output slots: the step's pools go to slots [first * m,
 // (first + count) * m).  Called by every lane of the warp; `stage` is 64
 // words of this warp's shared-memory scratch.  srow (optional) gets each
-// pool's score for each of its tokens.
+// pool's score for each of its tokens.  minv = ceil(2^32 / m): j / m is
+// umulhi(j, minv) for every j < count * m (j * m < 2^32).
 __device__ __forceinline__ void emit_expanded(bool keep, int pos, uint32_t key, uint32_t ix, int first, int count,
-                                              int m, int32_t* orow, float* srow, uint32_t* stage, int lane) {
+                                              int m, uint32_t minv, int32_t* orow, float* srow, uint32_t* stage,
+                                              int lane) {
   if (keep) {
     stage[pos - first] = ix;
     stage[32 + pos - first] = key;
   }
   __syncwarp();
   for (int j = lane; j < count * m; j += 32) {
-    const int e = j / m;
+    const int e = static_cast<int>(__umulhi(static_cast<uint32_t>(j), minv));
     orow[first * m + j] = static_cast<int32_t>(stage[e]) * m + (j - e * m);
     if (srow) srow[first * m + j] = key_to_float(stage[32 + e]);
   }
@@ -775,6 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->never, 1);
     bars->abort = 0;
     bars->tmem_busy = 0;
+    bars->cut_round = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -942,6 +953,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // NQW queries (all H heads of each)
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(eg * C::CW);
     uint32_t af_bits = 0u;  // phase parity of accumulator a's full barrier in bit a
+    // Cut rounds.  While one group cuts a buffer, the other groups soon stall
+    // (every group drains every tile), so a group whose buffer fills raises
+    // the CTA's round counter and the others, seeing it at their next tile,
+    // cut their fuller buffers at the same time: the cuts overlap instead of
+    // stalling the tensor core one after another.
+    // (bf16 variants; the FP8 ones keep the plain per-group cuts, which
+    // measured faster there)
+    constexpr bool kRounds = !FP8;
+    volatile int* cut_round = &bars->cut_round;
+    volatile int* seen = &bars->seen[eg];
     uint32_t tcount = 0;    // tiles drained so far; tile n sits in accumulator n & 1
     int par = 0;
     bool failed = false;
@@ -972,6 +993,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           st->pq[qi][c] = c < kPruneR ? 0.5f * v : v;  // kept-head weights halved, as for relu2
         }
       }
+      if (kRounds && etid == 0) *seen = *cut_round;
       if (etid < NQW) {
         const int64_t t = tq0 + etid;
         st->nvis[etid] = t < p.S ? n_visible(p, p.q_pos0 + t) : 0;
@@ -1017,7 +1039,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           thr_r[qi] = st->thr[qi];
           nvis_r[qi] = st->nvis[qi];
         }
-        bool any_full = false;
+        bool any_full = false, join = false;
         // per-key values of the next tile (FP8 key scale, pruning key norm),
         // loaded one tile ahead so that their latency hides behind the wait
         // for the accumulator and the head sums
@@ -1127,9 +1149,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             bals[qi] = __ballot_sync(kFullMask, pass);
             if (lane == 0) reinterpret_cast<int32_t*>(&st->wc[par][qi])[wq] = __popc(bals[qi]);
           }
-          if (named_bar_or(bar_id, kBM, !ok)) {
-            failed = true;
-            break;
+          // one barrier for two votes: a failed wait (every thread of the
+          // failing warp but etid 1, so at least 31) and a new cut round
+          // (etid 1 alone)
+          if constexpr (kRounds) {
+            const bool vote = etid == 1 ? (*cut_round != *seen) : !ok;
+            const uint32_t votes = named_bar_popc(bar_id, kBM, vote);
+            if (votes > 1u) {
+              failed = true;
+              break;
+            }
+            join = votes == 1u;
+          } else {
+            if (named_bar_or(bar_id, kBM, !ok)) {
+              failed = true;
+              break;
+            }
           }
           // ordered append: position = held + earlier warps + earlier lanes.  No
           // barrier follows: every thread knows the new counts, and the per-warp
@@ -1150,7 +1185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           par ^= 1;
 #pragma unroll
           for (int qi = 0; qi < NQW; ++qi) any_full |= held[qi] > p.cap - kBM;
-          if (any_full) {
+          if (any_full || join) {
             ++j;
             break;
           }
@@ -1159,15 +1194,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int qi = 0; qi < NQW; ++qi)
           if (etid == qi) st->cnt[par][qi] = held[qi];
-        // no buffer is full: the block's tiles are done and the final top-K of
-        // each query is written; otherwise the full buffers are cut back
-        const bool fin = !any_full;
+        // a cut round: this group's own buffer is full, or another group's
+        // round is joined; otherwise the block's tiles are done and the final
+        // top-K of each query is written
+        const bool fin = !(any_full || join);
+        if (kRounds && !fin && etid == 0) {
+          if (any_full) atomicAdd(const_cast<int*>(cut_round), 1);
+          *seen = *cut_round;
+        }
         named_bar(bar_id, kBM);  // every append and count of the last tile is visible to the group
+        // buffers fuller than this are cut in a round: every full one (held >
+        // cap - kBM >= cut_min) and those of the joining groups that are well
+        // on their way
+        const int cut_min = kRounds ? (p.cap + p.ksel) / 2 : p.cap - kBM;
 #pragma unroll 1
         for (int qi = 0; qi < NQW; ++qi) {
           const int n = st->cnt[par][qi];
           const int64_t t = tq0 + qi;
-          if (fin ? t >= p.S : n <= p.cap - kBM) continue;
+          if (fin ? t >= p.S : n <= cut_min) continue;
           if (!fin) {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
             int kept;
@@ -1196,6 +1240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int32_t* orow = p.out_idx + t * p.width;
             float* srow = p.out_score ? p.out_score + t * p.width : nullptr;
             const int m = p.out_ratio;
+            const uint32_t minv = p.out_ratio_inv;
             // with split key ranges this is one split's top-K, kept as
             // (ordered score, key) pairs in key order for the merge
             uint2* srow_split = nullptr;
@@ -1221,7 +1266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (SPLIT || m == 1) {
                 if (keep) emit(pos, k, ix);
               } else {
-                emit_expanded(keep, pos, k, ix, first, count, m, orow, srow, hist + (etid >> 5) * 64, etid & 31);
+                emit_expanded(keep, pos, k, ix, first, count, m, minv, orow, srow, hist + (etid >> 5) * 64,
+                              etid & 31);
               }
             };
             int kept;
