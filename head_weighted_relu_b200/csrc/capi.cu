@@ -108,7 +108,7 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
   pl->ranged = token ? 0 : 1;
   const int64_t nb = (p->S + pl->var.queries_per_block - 1) / pl->var.queries_per_block;
   pl->n_blocks = static_cast<int32_t>(nb);
-  pl->cap = candidate_capacity(pl->ksel);
+  pl->cap = candidate_capacity(pl->ksel, (p->flags & INDEXER_FLAG_PRUNE) != 0);
   pl->grid = 0;
   pl->cand_bytes = 0;
   pl->splits = 1;
@@ -135,7 +135,9 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
     }
     const int64_t items = nb * pl->splits;
     pl->grid = static_cast<int32_t>(items < di.sms ? items : di.sms);
-    pl->cand_bytes = static_cast<size_t>(pl->grid) * pl->var.groups * pl->var.queries_per_wg *
+    // two sets: a finished block's buffers are read by the row writers while
+    // the next block fills the other set
+    pl->cand_bytes = static_cast<size_t>(pl->grid) * 2 * pl->var.groups * pl->var.queries_per_wg *
                      static_cast<size_t>(pl->cap) * sizeof(uint2);
     if (pl->splits > 1) {
       pl->split_bytes = align256(static_cast<size_t>(p->S) * pl->splits * pl->ksel * sizeof(uint2));

@@ -68,14 +68,21 @@ struct ScoreVariant {
 bool score_variant(int H, int D, bool fp8, bool prune, ScoreVariant* out);
 
 // Candidate-buffer capacity per query for a selection budget of ksel keys.
-inline int candidate_capacity(int ksel) {
+inline int candidate_capacity(int ksel, bool prune) {
   // the budget plus as much again for new candidates, and up to four times the
-  // budget while that still fits the register-resident selection (4,096):
-  // fewer cuts for small budgets
+  // budget (eight without the pruning certificate) while that still fits the
+  // register-resident selection (4,096): fewer cuts for small budgets.  With
+  // pruning a smaller buffer fills, and so raises the running threshold the
+  // certificate screens against, sooner on short rows.
   auto r128 = [](int x) { return ((x + 127) / 128) * 128; };
   int c = r128(2 * ksel);
-  const int wide = r128(4 * ksel);
-  if (wide <= 4096 && wide > c) c = wide;
+  if (prune) {
+    const int wide = r128(4 * ksel);
+    if (wide <= 4096 && wide > c) c = wide;
+  } else {
+    const int wide = r128(8 * ksel) < 4096 ? r128(8 * ksel) : 4096;
+    if (wide > c) c = wide;
+  }
   return c < ksel + 256 ? r128(ksel + 256) : c;
 }
 

@@ -62,6 +62,10 @@ constexpr int kDigitBits = 10;                   // radix digit width
 constexpr int kHistBins = 1 << kDigitBits;
 constexpr int kSmemLimit = 232448;               // 227 KB opt-in shared memory per CTA
 constexpr uint64_t kWaitLimitNs = 4000000000ull; // give up a pipeline wait after 4 s
+// Final hand-off: what the writer warps do with one query's candidate buffer.
+constexpr uint32_t kJobSkip = 0;   // no such query row (past the last)
+constexpr uint32_t kJobAll = 1;    // every entry is kept (at most K of them)
+constexpr uint32_t kJobCut = 2;    // keep e.x > v, or e.x == v and e.y <= icut
 
 template <int NQ>
 struct WgState {
@@ -92,6 +96,14 @@ struct Barriers {
   int tmem_busy;       // MMAs may still write TMEM: leave it allocated
   int cut_round;       // raised by a group whose buffer filled: others cut too
   int seen[4];         // the cut round each epilogue group has taken part in
+  // Final hand-off (single-range kernel): candidate buffers alternate between
+  // two sets by the CTA's block count; a group posts its block's cuts to set
+  // s and arrives on fin_full[s] (4 arrivals), the two writer warps write the
+  // output rows and arrive on fin_free[s] (2 arrivals) once they are done
+  // with the set's buffers.
+  uint64_t fin_full[2], fin_free[2];
+  uint4 jobs[2][4][8];       // [set][group][query]: n, v, icut, mode (kJob*)
+  uint32_t fstage[2][64];    // per writer warp: kept pools of one step (pool expansion)
 };
 
 template <int H, int D, bool FP8>
@@ -138,7 +150,8 @@ struct Cfg {
   static_assert(STAGES >= 2, "shared memory too small for a 2-stage key ring");
   static_assert(SMEM_BYTES <= kSmemLimit, "shared memory");
   static_assert(OFF_K % 1024 == 0 && K_STAGE_BYTES % 1024 == 0 && Q_ACC_BYTES % 1024 == 0, "swizzle alignment");
-  static_assert(OFF_BAR % 8 == 0 && OFF_ST % 16 == 0 && OFF_W % 16 == 0, "alignment");
+  static_assert(OFF_BAR % 16 == 0 && OFF_ST % 16 == 0 && OFF_W % 16 == 0, "alignment");
+  static_assert(NQW <= 8, "final hand-off slots");
 };
 
 __device__ __forceinline__ int32_t n_visible(const ScoreParams& p, int64_t g) {
@@ -744,6 +757,71 @@ __device__ __forceinline__ void emit_expanded(bool keep, int pos, uint32_t key, 
   __syncwarp();
 }
 
+// The output row of query t, written by one warp from the query's candidate
+// buffer (entries in key order) and the cut its group computed (`job`): the
+// kept keys in key order ("Adjacent-Query KV-Index Overlap in 256K DSA
+// Training", §3), each pool expanded to its token positions and the
+// incomplete pool's positions appended ("Module 06 — DSA & KPool", §2), then
+// -1 padding and the valid length.  Entries are read two warp-steps at a time
+// so that two loads are in flight.  `stage` is 64 words of this warp's
+// shared memory.
+__device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScoreParams& p, int64_t t,
+                                      uint32_t* stage, int lane) {
+  const int n = static_cast<int>(job.x);
+  const bool all = job.w == kJobAll;
+  const uint32_t v = all ? 0u : job.y;
+  const uint32_t icut = all ? 0xFFFFFFFFu : job.z;
+  const int m = p.out_ratio;
+  int32_t* orow = p.out_idx + t * p.width;
+  float* srow = p.out_score ? p.out_score + t * p.width : nullptr;
+  const uint32_t lt = (1u << lane) - 1u;
+  int kept = 0;
+  for (int i0 = 0; i0 < n; i0 += 2 * 32) {
+    uint2 e[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * 32 + lane;
+      e[u] = i < n ? buf[i] : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * 32 + lane;
+      const bool keep = (i < n) & ((e[u].x > v) | ((e[u].x == v) & (e[u].y <= icut)));
+      const uint32_t bal = __ballot_sync(kFullMask, keep);
+      const int pos = kept + __popc(bal & lt);
+      if (m == 1) {
+        if (keep) {
+          orow[pos] = static_cast<int32_t>(e[u].y);
+          if (srow) srow[pos] = key_to_float(e[u].x);
+        }
+      } else if (bal != 0u) {
+        emit_expanded(keep, pos, e[u].x, e[u].y, kept, __popc(bal), m, p.out_ratio_inv, orow, srow, stage, lane);
+      }
+      kept += __popc(bal);
+    }
+  }
+  int len = kept * m;
+  if (m > 1) {
+    const int64_t g = p.q_pos0 + t;
+    const int tail = static_cast<int>((g + 1) % m);
+    const int64_t first = g + 1 - tail;
+    for (int i = lane; i < tail; i += 32) {
+      orow[len + i] = static_cast<int32_t>(first + i);
+      if (srow) srow[len + i] = __uint_as_float(0x7FC00000u);
+    }
+    len += tail;
+  }
+  for (int i = len + lane; i < p.width; i += 32) {
+    orow[i] = -1;
+    if (srow) srow[i] = __uint_as_float(0x7FC00000u);
+  }
+  if (lane == 0) {
+    p.out_len[t] = len;
+    // with a seed threshold at least min(K, visible) keys must pass it
+    if (p.seed_thr != nullptr && kept < min(p.ksel, n_visible(p, p.q_pos0 + t))) atomicOr(p.status, kStatusWitness);
+  }
+}
+
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
@@ -783,6 +861,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->never, 1);
+    for (int f = 0; f < 2; ++f) {
+      mbar_init(&bars->fin_full[f], kEpiGroups);  // one arrival per epilogue group
+      mbar_init(&bars->fin_free[f], 2);           // one per writer warp
+    }
     bars->abort = 0;
     bars->tmem_busy = 0;
     bars->cut_round = 0;
@@ -921,6 +1003,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         bars->tmem_busy = 1;
       }
     }
+  } else if constexpr (!SPLIT && !FP8) {
+    // ---------------------------------------------------- output-row writers
+    // Warps 2 and 3 write the output rows of each finished query block while
+    // the epilogue groups go on with the next block: a group hands over its
+    // queries' candidate buffers (one of two sets) with their final cuts.
+    const int ww = warp - 2;
+    for (int r = 0;; ++r) {
+      const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+      if (it.b < 0) break;
+      const int set = r & 1;
+      bool ok = mbar_wait(&bars->fin_full[set], static_cast<uint32_t>(r >> 1) & 1u, abort_flag, kWaitLimitNs);
+      if (!__any_sync(kFullMask, ok)) {
+        if (lane == 0) {
+          atomicOr(p.status, kStatusWaitTimeout);
+          bars->abort = 1;
+        }
+        break;
+      }
+      for (int jb = ww; jb < kEpiGroups * NQW; jb += 2) {
+        const int g = jb / NQW, qi = jb - g * NQW;
+        const uint4 job = bars->jobs[set][g][qi];
+        if (job.w == kJobSkip) continue;
+        const int64_t t = static_cast<int64_t>(it.b) * QB + g * NQW + qi;
+        const uint2* buf = p.cand + ((static_cast<size_t>(blockIdx.x) * 2 + set) * kEpiGroups + g) * NQW *
+                                        static_cast<size_t>(p.cap) +
+                           qi * static_cast<size_t>(p.cap);
+        warp_write_row(buf, job, p, t, bars->fstage[ww], lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->fin_free[set]);
+    }
   }
   __syncwarp();  // lane 0 of warps 0 and 1 rejoins its warp before the aligned barrier
   tc_fence_before();
@@ -961,6 +1074,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (bf16 variants; the FP8 ones keep the plain per-group cuts, which
     // measured faster there)
     constexpr bool kRounds = !FP8;
+    // The single-range bf16 kernels hand each finished block's output rows to
+    // the writer warps (warps 2 and 3) and go on with the next block; the
+    // split-range kernel writes its per-range lists itself, and the FP8 kernel
+    // (long rows, few blocks, the most register-bound epilogue) its rows.
+    constexpr bool kDefer = !SPLIT && !FP8;
     volatile int* cut_round = &bars->cut_round;
     volatile int* seen = &bars->seen[eg];
     uint32_t tcount = 0;    // tiles drained so far; tile n sits in accumulator n & 1
@@ -973,9 +1091,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (b < 0) break;
       const int nt = it.j1;
       const int64_t tq0 = static_cast<int64_t>(b) * QB + eg * NQW;
-      uint2* cand = p.cand + (static_cast<size_t>(blockIdx.x) * kEpiGroups + eg) * NQW * static_cast<size_t>(p.cap);
-
-      named_bar(bar_id, kBM);  // the previous block is completely done with the state
+      const int set = r & 1;  // candidate-buffer set of this block
+      uint2* cand = p.cand + ((static_cast<size_t>(blockIdx.x) * 2 + set) * kEpiGroups + eg) * NQW *
+                                 static_cast<size_t>(p.cap);
+      bool free_ok = true;
+      if (kDefer && r >= 2) {
+        // the writer warps are done with this set's buffers (block r - 2)
+        free_ok = mbar_wait(&bars->fin_free[set], static_cast<uint32_t>((r >> 1) - 1) & 1u, abort_flag,
+                            kWaitLimitNs);
+        free_ok = __any_sync(kFullMask, free_ok);
+      }
+      // the previous block is completely done with the state
+      if (named_bar_or(bar_id, kBM, !free_ok)) {
+        failed = true;
+        break;
+      }
       for (int i = etid; i < C::CW; i += kBM) {
         const int64_t t = tq0 + i / H;
         float v = 0.f;
@@ -1211,6 +1341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int qi = 0; qi < NQW; ++qi) {
           const int n = st->cnt[par][qi];
           const int64_t t = tq0 + qi;
+          if (kDefer && fin && etid == 0 && t >= p.S) bars->jobs[set][eg][qi] = make_uint4(0u, 0u, 0u, kJobSkip);
           if (fin ? t >= p.S : n <= cut_min) continue;
           if (!fin) {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
@@ -1234,6 +1365,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               st->cnt[par][qi] = kept;
               st->thr[qi] = thr;
             }
+          } else if constexpr (kDefer) {
+            // the cut only: the writer warps write the row
+            uint2* buf = cand + qi * static_cast<size_t>(p.cap);
+            uint4 job = make_uint4(static_cast<uint32_t>(n), 0u, 0xFFFFFFFFu, kJobAll);
+            if (n > p.ksel) {
+              if (n <= kRegCap) {
+                RegBuf rb;
+                rb_load(rb, buf, n, etid);
+                const RegCut c = rb_cut(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist, st->red, etid, bar_id);
+                job = make_uint4(static_cast<uint32_t>(n), c.v, c.icut, kJobCut);
+              } else {
+                const Cut c = wg_topk_cut(buf, n, static_cast<uint32_t>(p.ksel), hist, st->red, etid, bar_id);
+                job = make_uint4(static_cast<uint32_t>(n), c.v, c.icut, kJobCut);
+              }
+            }
+            if (etid == 0) bars->jobs[set][eg][qi] = job;
           } else {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
             const bool all = n <= p.ksel;
@@ -1332,7 +1479,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           named_bar(bar_id, kBM);
         }
-        if (fin) break;
+        if (fin) {
+          // every cut of the block is posted (and the last tile's appends are
+          // visible to the group): hand the block to the writer warps
+          if (kDefer && etid == 0) mbar_arrive(&bars->fin_full[set]);
+          break;
+        }
       }
     }
     if (failed && etid == 0) {
