@@ -73,7 +73,7 @@ struct WgState {
   int32_t cnt[2][NQ];    // candidates held, double-buffered by tile parity
   int32_t nvis[NQ];      // keys visible to each query of the group
   int4 wc[2][NQ];        // per-warp pass counts (x..w = warps 0..3), double-buffered by tile parity
-  uint32_t red[16];      // reduction scratch
+  uint32_t red[24];      // reduction scratch
   int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
   int32_t scan[4];       // per-warp totals of a register-resident compaction
   // pruning: folded weights of the kept heads, then Ceff (read as float4)
@@ -493,9 +493,13 @@ struct Digit {
 // distinct banks), a suffix scan over the lanes finds the lane holding the
 // rank-th largest, a second scan over that lane's bins finds the digit, and
 // the warp clears the bins.  Two barriers.
+__device__ inline Digit rb_find_digit(int nb, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id);
+
+// (entries above `top` are left out: they lie in higher bins of an earlier
+// pass)
 __device__ inline Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t base,
-                         int shift, int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
-  const int lane = etid & 31, wq = etid >> 5;
+                         int shift, int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id,
+                         uint32_t top = 0xFFFFFFFFu) {
   const int nb = 1 << width;
   const unsigned long long span = 1ull << (shift + width);
   const int room = rb_room(n, etid);
@@ -504,9 +508,16 @@ __device__ inline Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool fil
     const uint32_t f = rb_field(b, r, idx_field);
     // branch-free: every condition is a predicate
     const bool ok = (32 * r < room) & (!filt | (b.key[r] == fval)) & (f >= base) &
-                    (static_cast<unsigned long long>(f - base) < span);
+                    (static_cast<unsigned long long>(f - base) < span) & (f <= top);
     if (ok) atomicAdd(&hist[(f - base) >> shift], 1u);
   }
+  return rb_find_digit(nb, rank, hist, red, etid, bar_id);
+}
+
+// The digit of a filled histogram (2^width = nb bins, counted from the top)
+// that holds the rank-th largest entry; clears the bins.  Two barriers.
+__device__ inline Digit rb_find_digit(int nb, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
+  const int lane = etid & 31, wq = etid >> 5;
   named_bar(bar_id, kBM);
   if (wq == 0) {
     const int per = nb >= 32 ? nb >> 5 : 1;   // bins per lane (a power of two)
@@ -580,16 +591,16 @@ __device__ __forceinline__ void warp_sort64_desc(unsigned long long (&v)[2], int
 }
 
 // The cut when the remaining candidates -- the entries whose ordered score
-// lies in [base, base + 2^shift) -- number at most kSmallSel: they are
+// lies in [base, base + span) -- number at most kSmallSel: they are
 // gathered into shared memory (hist[512, 640), free after the passes), warp
 // 0 sorts them by (ordered score desc, index asc) and the rank-th of them
 // gives v and the index cut.  red[12] counts the gathered entries (cleared by
 // the caller before its first barrier).
-__device__ inline RegCut rb_small_select(const RegBuf& b, int n, uint32_t base, int shift, uint32_t rank,
-                                         uint32_t ksel, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
+__device__ inline RegCut rb_small_select(const RegBuf& b, int n, uint32_t base, unsigned long long span,
+                                         uint32_t rank, uint32_t ksel, uint32_t* hist, uint32_t* red, int etid,
+                                         int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
   const int room = rb_room(n, etid);
-  const unsigned long long span = 1ull << shift;
   uint2* list = reinterpret_cast<uint2*>(hist + 512);
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r) {
@@ -619,13 +630,60 @@ __device__ inline RegCut rb_small_select(const RegBuf& b, int n, uint32_t base, 
   return {red[8], red[9], false, static_cast<int>(ksel)};
 }
 
+// Bin of an entry in a first pass linear in the score value: 1,024 bins over
+// [fmn, fmn + 1024 / scale].  Rounded subtraction, multiplication by a
+// positive scale and truncation are each monotone, so a higher bin holds only
+// strictly higher scores and equal scores share a bin.
+__device__ __forceinline__ uint32_t score_bin(uint32_t key, float fmn, float scale) {
+  return min(static_cast<uint32_t>(kHistBins - 1), __float2uint_rz((key_to_float(key) - fmn) * scale));
+}
+
+// First pass over score values: the bin holding the rank-th largest entry.
+__device__ inline Digit rb_fpass(const RegBuf& b, int n, float fmn, float scale, uint32_t rank, uint32_t* hist,
+                                 uint32_t* red, int etid, int bar_id) {
+  const int room = rb_room(n, etid);
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r)
+    if (32 * r < room) atomicAdd(&hist[score_bin(b.key[r], fmn, scale)], 1u);
+  return rb_find_digit(kHistBins, rank, hist, red, etid, bar_id);
+}
+
+// Smallest and largest ordered score among the entries of first-pass bin d
+// (the bin is not empty).  One barrier; `red` is reused by the next phase
+// only after its own barrier.
+__device__ inline void rb_bin_range(const RegBuf& b, int n, float fmn, float scale, uint32_t d, uint32_t& lo,
+                                    uint32_t& hi, uint32_t* red, int etid, int bar_id) {
+  const int lane = etid & 31, wq = etid >> 5;
+  const int room = rb_room(n, etid);
+  uint32_t mx = 0u, mn = 0xFFFFFFFFu;
+#pragma unroll
+  for (int r = 0; r < kRegEntries; ++r) {
+    const uint32_t k = b.key[r];
+    const bool in = (32 * r < room) & (score_bin(k, fmn, scale) == d);
+    mx = max(mx, in ? k : 0u);
+    mn = min(mn, in ? k : 0xFFFFFFFFu);
+  }
+  mx = warp_max_u32(mx);
+  mn = warp_min_u32(mn);
+  if (lane == 0) {
+    red[16 + wq] = mx;
+    red[20 + wq] = mn;
+  }
+  named_bar(bar_id, kBM);
+  hi = max(max(red[16], red[17]), max(red[18], red[19]));
+  lo = min(min(red[20], red[21]), min(red[22], red[23]));
+}
+
 // Radix select of the ksel-th largest (ordered score, then lowest index).
-// Passes of up to 10 bits walk down from the span [min, max] of the scores:
-// each pass narrows the range holding the ksel-th entry to one bin.  With
-// `approx`, stops after the first pass if keeping everything from that bin up
-// keeps at most `room` entries: a safe lower bound for a running threshold.
-// Once the bin holding the ksel-th entry has at most kSmallSel entries, they
-// are sorted in one warp (rb_small_select) instead of further passes.
+// The first pass puts the scores into 1,024 bins linear in their value (a
+// pass on the bits of the ordered score would put most of a score
+// distribution into the few bins of one or two binary exponents); later
+// passes of up to 10 bits walk down the ordered scores of the bin holding
+// the ksel-th entry.  With `approx`, stops after the first pass if keeping
+// everything from that bin up keeps at most `room` entries: a safe lower
+// bound for a running threshold.  Once the bin holding the ksel-th entry has
+// at most kSmallSel entries, they are sorted in one warp (rb_small_select)
+// instead of further passes.
 __device__ inline RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int room, uint32_t* hist,
                          uint32_t* red, int etid, int bar_id) {
   uint32_t mx, mn;
@@ -637,28 +695,46 @@ __device__ inline RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool appr
   rb_maxmin(b, n, false, false, 0u, mx, mn, red, etid, bar_id);
   uint32_t base = mn, above = 0u, cnt = static_cast<uint32_t>(n), rank = ksel;
   if (mx != mn) {
-    int shift = 32 - __clz(mx - mn);  // bits of the span of the scores
-    bool first = true;
-    while (shift > 0) {
-      const int width = shift < kDigitBits ? shift : kDigitBits;
-      shift -= width;
-      const Digit dg = rb_pass(b, n, false, false, 0u, base, shift, width, rank, hist, red, etid, bar_id);
-      base += dg.d << shift;
-      above += dg.above;
-      rank -= dg.above;
-      cnt = dg.cnt;
-      if (approx && first && static_cast<int>(above + cnt) <= room)
-        return {base, 0u, true, static_cast<int>(above + cnt)};
-      first = false;
-      if (cnt <= static_cast<uint32_t>(kSmallSel))
-        return rb_small_select(b, n, base, shift, rank, ksel, hist, red, etid, bar_id);
+    const float fmn = key_to_float(mn);
+    float scale = static_cast<float>(kHistBins) / (key_to_float(mx) - fmn);
+    if (!(scale < 1.0e30f)) scale = 0.f;  // a span too narrow for float bins: one bin, passes below
+    const Digit d0 = rb_fpass(b, n, fmn, scale, rank, hist, red, etid, bar_id);
+    above += d0.above;
+    rank -= d0.above;
+    cnt = d0.cnt;
+    uint32_t lo, hi;
+    rb_bin_range(b, n, fmn, scale, d0.d, lo, hi, red, etid, bar_id);
+    // every entry of a higher bin scores above hi, every entry of a lower
+    // one below lo: [lo, hi] holds exactly the bin's entries
+    if (approx && static_cast<int>(above + cnt) <= room) return {lo, 0u, true, static_cast<int>(above + cnt)};
+    if (cnt <= static_cast<uint32_t>(kSmallSel))
+      return rb_small_select(b, n, lo, static_cast<unsigned long long>(hi - lo) + 1ull, rank, ksel, hist, red,
+                             etid, bar_id);
+    base = lo;
+    if (hi != lo) {
+      int shift = 32 - __clz(hi - lo);  // bits of the bin's span of ordered scores
+      while (shift > 0) {
+        const int width = shift < kDigitBits ? shift : kDigitBits;
+        shift -= width;
+        const Digit dg = rb_pass(b, n, false, false, 0u, base, shift, width, rank, hist, red, etid, bar_id, hi);
+        base += dg.d << shift;
+        above += dg.above;
+        rank -= dg.above;
+        cnt = dg.cnt;
+        if (cnt <= static_cast<uint32_t>(kSmallSel)) {
+          const unsigned long long digit_span = 1ull << shift;
+          const unsigned long long to_hi = static_cast<unsigned long long>(hi - base) + 1ull;
+          return rb_small_select(b, n, base, digit_span < to_hi ? digit_span : to_hi, rank, ksel, hist, red,
+                                 etid, bar_id);
+        }
+      }
     }
   }
   // base is now v, the ksel-th largest ordered score; `rank` of the `cnt`
   // entries tied at v make the cut
   if (rank >= cnt) return {base, 0xFFFFFFFFu, false, static_cast<int>(above + cnt)};
   if (cnt <= static_cast<uint32_t>(kSmallSel))
-    return rb_small_select(b, n, base, 0, rank, ksel, hist, red, etid, bar_id);
+    return rb_small_select(b, n, base, 1ull, rank, ksel, hist, red, etid, bar_id);
   // many ties at v: the rank-th largest ~index among them, by the same passes
   const uint32_t v = base;
   uint32_t imx, imn;

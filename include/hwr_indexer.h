@@ -172,7 +172,7 @@ indexer_status indexer_topk(const indexer_problem* p,
  *   every GPU that loads the library holds until the process exits.
  *   Problems whose indexer_workspace_bytes exceeds 64 MiB are rejected with
  *   INDEXER_EWORKSPACE before anything is launched (on a 148-SM B200 with
- *   H = 64 that allows budgets up to K = 7,040).
+ *   H = 64 that allows budgets up to K = 3,520).
  *   The first call on each device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
  *   Nothing here allocates.  All calls share the one array and it keeps the
