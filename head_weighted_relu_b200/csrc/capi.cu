@@ -135,9 +135,9 @@ indexer_status make_plan(const indexer_problem* p, bool need_device, Plan* pl) {
     }
     const int64_t items = nb * pl->splits;
     pl->grid = static_cast<int32_t>(items < di.sms ? items : di.sms);
-    // two sets: a finished block's buffers are read by the row writers while
-    // the next block fills the other set
-    pl->cand_bytes = static_cast<size_t>(pl->grid) * 2 * pl->var.groups * pl->var.queries_per_wg *
+    // kCandSets sets: a finished block's buffers are read by the row writers
+    // while the next blocks fill the other sets
+    pl->cand_bytes = static_cast<size_t>(pl->grid) * kCandSets * pl->var.groups * pl->var.queries_per_wg *
                      static_cast<size_t>(pl->cap) * sizeof(uint2);
     if (pl->splits > 1) {
       pl->split_bytes = align256(static_cast<size_t>(p->S) * pl->splits * pl->ksel * sizeof(uint2));

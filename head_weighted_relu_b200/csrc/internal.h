@@ -13,6 +13,10 @@ constexpr uint32_t kStatusWaitTimeout = 1u;
 constexpr uint32_t kStatusOverflow = 2u;
 constexpr uint32_t kStatusWitness = 4u;  // a seed threshold left a query fewer than min(K, visible) keys
 
+// Candidate-buffer sets per CTA and epilogue group (the scoring kernel's
+// kSets): blocks rotate through them while the row writers read finished ones.
+constexpr int kCandSets = 3;
+
 // Heads the pruning certificate keeps exactly (the first kPruneR of each query).
 constexpr int kPruneR = 16;
 

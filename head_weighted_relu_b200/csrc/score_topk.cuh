@@ -62,6 +62,9 @@ constexpr int kDigitBits = 10;                   // radix digit width
 constexpr int kHistBins = 1 << kDigitBits;
 constexpr int kSmemLimit = 232448;               // 227 KB opt-in shared memory per CTA
 constexpr uint64_t kWaitLimitNs = 4000000000ull; // give up a pipeline wait after 4 s
+// Candidate-buffer sets: a block's buffers are read by the row writers while
+// the groups fill the next sets (block r uses set r % kSets).
+constexpr int kSets = kCandSets;
 // Final hand-off: what the writer warps do with one query's candidate buffer.
 constexpr uint32_t kJobSkip = 0;   // no such query row (past the last)
 constexpr uint32_t kJobAll = 1;    // every entry is kept (at most K of them)
@@ -88,7 +91,7 @@ struct Barriers {
   uint64_t kfull[STAGES];
   uint64_t kempty[STAGES];
   uint64_t qfull, qempty;
-  uint64_t accfull[2], accempty[2];
+  uint64_t accfull[4], accempty[4];
   uint64_t mma_done;
   uint64_t never;      // test hook: a barrier nothing arrives at
   uint32_t tmem_slot;
@@ -96,13 +99,13 @@ struct Barriers {
   int tmem_busy;       // MMAs may still write TMEM: leave it allocated
   int cut_round;       // raised by a group whose buffer filled: others cut too
   int seen[4];         // the cut round each epilogue group has taken part in
-  // Final hand-off (single-range kernel): candidate buffers alternate between
-  // two sets by the CTA's block count; a group posts its block's cuts to set
-  // s and arrives on fin_full[s] (4 arrivals), the two writer warps write the
-  // output rows and arrive on fin_free[s] (2 arrivals) once they are done
+  // Final hand-off (single-range kernel): candidate buffers rotate through
+  // kSets sets by the CTA's block count; a group posts its block's cuts to
+  // set s and arrives on fin_full[s] (4 arrivals), the two writer warps write
+  // the output rows and arrive on fin_free[s] (2 arrivals) once they are done
   // with the set's buffers.
-  uint64_t fin_full[2], fin_free[2];
-  uint4 jobs[2][4][8];       // [set][group][query]: n, v, icut, mode (kJob*)
+  uint64_t fin_full[kSets], fin_free[kSets];
+  uint4 jobs[kSets][4][8];   // [set][group][query]: n, v, icut, mode (kJob*)
   uint32_t fstage[2][64];    // per writer warp: kept pools of one step (pool expansion)
 };
 
@@ -129,7 +132,10 @@ struct Cfg {
   static constexpr int Q_ACC_BYTES = BN * ROW_BYTES;
   static constexpr int Q_BYTES = Q_ACC_BYTES;
   static constexpr int K_STAGE_BYTES = kBM * ROW_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;
+  // accumulators: as many as TMEM's 512 columns hold (2 at N = 256, 4 at
+  // N = 128); key tile n goes to accumulator n % NACC
+  static constexpr int NACC = 512 / BN;
+  static constexpr int TMEM_COLS = NACC * BN;
   static constexpr int SMALL_BYTES =
       kHistBins * 4 * kEpiGroups + BN * 4 + kEpiGroups * (int)sizeof(WgState<NQW>);
   static constexpr int AVAIL = kSmemLimit - 1024 - Q_BYTES - SMALL_BYTES - (int)sizeof(Barriers<8>);
@@ -931,13 +937,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->qfull, 1);
     mbar_init(&bars->qempty, 1);
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < 4; ++a) {
       mbar_init(&bars->accfull[a], 1);
       mbar_init(&bars->accempty[a], 16);  // one arrival per epilogue warp
     }
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->never, 1);
-    for (int f = 0; f < 2; ++f) {
+    for (int f = 0; f < kSets; ++f) {
       mbar_init(&bars->fin_full[f], kEpiGroups);  // one arrival per epilogue group
       mbar_init(&bars->fin_free[f], 2);           // one per writer warp
     }
@@ -1018,7 +1024,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t k_base = smem_u32(smem + C::OFF_K);
       int stage = 0;
       uint32_t kph = 0, qf_ph = 0;
-      uint32_t ae_ph[2] = {0u, 0u};
+      uint32_t ae_ph[4] = {0u, 0u, 0u, 0u};
       uint32_t tcount = 0;  // tiles issued so far; tile n goes to accumulator n & 1
       bool ok = true;
       for (int r = 0; ok; ++r) {
@@ -1034,7 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t kst = k_base + stage * C::K_STAGE_BYTES;
-          const int a = static_cast<int>(tcount & 1u);
+          const int a = static_cast<int>(tcount % C::NACC);
           ok = mbar_wait(&bars->accempty[a], ae_ph[a] ^ 1u, abort_flag, kWaitLimitNs);
           ae_ph[a] ^= 1u;
           if (!ok) break;
@@ -1088,8 +1094,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int r = 0;; ++r) {
       const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
       if (it.b < 0) break;
-      const int set = r & 1;
-      bool ok = mbar_wait(&bars->fin_full[set], static_cast<uint32_t>(r >> 1) & 1u, abort_flag, kWaitLimitNs);
+      const int set = r % kSets;
+      bool ok = mbar_wait(&bars->fin_full[set], static_cast<uint32_t>(r / kSets) & 1u, abort_flag, kWaitLimitNs);
       if (!__any_sync(kFullMask, ok)) {
         if (lane == 0) {
           atomicOr(p.status, kStatusWaitTimeout);
@@ -1102,7 +1108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint4 job = bars->jobs[set][g][qi];
         if (job.w == kJobSkip) continue;
         const int64_t t = static_cast<int64_t>(it.b) * QB + g * NQW + qi;
-        const uint2* buf = p.cand + ((static_cast<size_t>(blockIdx.x) * 2 + set) * kEpiGroups + g) * NQW *
+        const uint2* buf = p.cand + ((static_cast<size_t>(blockIdx.x) * kSets + set) * kEpiGroups + g) * NQW *
                                         static_cast<size_t>(p.cap) +
                            qi * static_cast<size_t>(p.cap);
         warp_write_row(buf, job, p, t, bars->fstage[ww], lane);
@@ -1167,13 +1173,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (b < 0) break;
       const int nt = it.j1;
       const int64_t tq0 = static_cast<int64_t>(b) * QB + eg * NQW;
-      const int set = r & 1;  // candidate-buffer set of this block
-      uint2* cand = p.cand + ((static_cast<size_t>(blockIdx.x) * 2 + set) * kEpiGroups + eg) * NQW *
+      const int set = r % kSets;  // candidate-buffer set of this block
+      uint2* cand = p.cand + ((static_cast<size_t>(blockIdx.x) * kSets + set) * kEpiGroups + eg) * NQW *
                                  static_cast<size_t>(p.cap);
       bool free_ok = true;
-      if (kDefer && r >= 2) {
-        // the writer warps are done with this set's buffers (block r - 2)
-        free_ok = mbar_wait(&bars->fin_free[set], static_cast<uint32_t>((r >> 1) - 1) & 1u, abort_flag,
+      if (kDefer && r >= kSets) {
+        // the writer warps are done with this set's buffers (block r - kSets)
+        free_ok = mbar_wait(&bars->fin_free[set], static_cast<uint32_t>(r / kSets - 1) & 1u, abort_flag,
                             kWaitLimitNs);
         free_ok = __any_sync(kFullMask, free_ok);
       }
@@ -1256,7 +1262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (PRUNE) kn_next = (j < nt && key < p.n_keys) ? p.knorm[key] : 0.f;
         }
         for (; j < nt; ++j) {
-          const int a = static_cast<int>(tcount & 1u);
+          const int a = static_cast<int>(tcount % C::NACC);
           ++tcount;
           const int32_t key = j * kBM + etid;
           const float ks = ks_next, kn = kn_next;
