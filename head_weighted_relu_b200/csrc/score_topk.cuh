@@ -833,7 +833,7 @@ __device__ __forceinline__ void emit_expanded(bool keep, int pos, uint32_t key, 
   __syncwarp();
   for (int j = lane; j < count * m; j += 32) {
     const int e = static_cast<int>(__umulhi(static_cast<uint32_t>(j), minv));
-    orow[first * m + j] = static_cast<int32_t>(stage[e]) * m + (j - e * m);
+    __stcs(&orow[first * m + j], static_cast<int32_t>(stage[e]) * m + (j - e * m));
     if (srow) srow[first * m + j] = key_to_float(stage[32 + e]);
   }
   __syncwarp();
@@ -873,7 +873,7 @@ __device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScorePa
       const int pos = kept + __popc(bal & lt);
       if (m == 1) {
         if (keep) {
-          orow[pos] = static_cast<int32_t>(e[u].y);
+          __stcs(&orow[pos], static_cast<int32_t>(e[u].y));
           if (srow) srow[pos] = key_to_float(e[u].x);
         }
       } else if (bal != 0u) {
@@ -888,13 +888,13 @@ __device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScorePa
     const int tail = static_cast<int>((g + 1) % m);
     const int64_t first = g + 1 - tail;
     for (int i = lane; i < tail; i += 32) {
-      orow[len + i] = static_cast<int32_t>(first + i);
+      __stcs(&orow[len + i], static_cast<int32_t>(first + i));
       if (srow) srow[len + i] = __uint_as_float(0x7FC00000u);
     }
     len += tail;
   }
   for (int i = len + lane; i < p.width; i += 32) {
-    orow[i] = -1;
+    __stcs(&orow[i], -1);
     if (srow) srow[i] = __uint_as_float(0x7FC00000u);
   }
   if (lane == 0) {
@@ -973,6 +973,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
+      // q rows are read once; key tiles are read by every CTA: keep the keys
+      // (and the candidate buffers) in L2 ahead of the q stream
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_k = l2_policy_evict_last();
       int stage = 0;
       uint32_t kph = 0, qe_ph = 0;
       bool first = true, ok = true;
@@ -994,7 +998,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->qfull, C::Q_BYTES);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_2d(smem + C::OFF_Q + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS, b * QB * H, &bars->qfull);
+          tma_load_2d_hint(smem + C::OFF_Q + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS, b * QB * H, &bars->qfull, pol_q);
         for (int j = it.j0; j < it.j1; ++j) {
           ok = mbar_wait(&bars->kempty[stage], kph ^ 1u, abort_flag, kWaitLimitNs);
           if (!ok) break;
@@ -1002,8 +1006,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&bars->kfull[stage], C::K_STAGE_BYTES);
 #pragma unroll
           for (int bx = 0; bx < C::NBOX; ++bx)
-            tma_load_2d(smem + C::OFF_K + stage * C::K_STAGE_BYTES + bx * kBM * 128, &tm_k, bx * C::BOX_ELEMS,
-                        j * kBM, &bars->kfull[stage]);
+            tma_load_2d_hint(smem + C::OFF_K + stage * C::K_STAGE_BYTES + bx * kBM * 128, &tm_k, bx * C::BOX_ELEMS,
+                             j * kBM, &bars->kfull[stage], pol_k);
           if (++stage == STAGES) {
             stage = 0;
             kph ^= 1u;
@@ -1481,11 +1485,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               const float sc = key_to_float(k);
               if (m == 1) {
-                orow[pos] = static_cast<int32_t>(ix);
+                __stcs(&orow[pos], static_cast<int32_t>(ix));
                 if (srow) srow[pos] = sc;
               } else {
                 for (int rr = 0; rr < m; ++rr) {
-                  orow[pos * m + rr] = static_cast<int32_t>(ix) * m + rr;
+                  __stcs(&orow[pos * m + rr], static_cast<int32_t>(ix) * m + rr);
                   if (srow) srow[pos * m + rr] = sc;
                 }
               }
@@ -1544,13 +1548,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int tail = static_cast<int>((g + 1) % m);
               const int64_t first = g + 1 - tail;
               for (int i = etid; i < tail; i += kBM) {
-                orow[len + i] = static_cast<int32_t>(first + i);
+                __stcs(&orow[len + i], static_cast<int32_t>(first + i));
                 if (srow) srow[len + i] = __uint_as_float(0x7FC00000u);
               }
               len += tail;
             }
             for (int i = len + etid; i < p.width; i += kBM) {
-              orow[i] = -1;
+              __stcs(&orow[i], -1);
               if (srow) srow[i] = __uint_as_float(0x7FC00000u);
             }
             if (etid == 0) {
