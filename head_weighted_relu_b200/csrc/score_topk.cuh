@@ -76,7 +76,8 @@ struct WgState {
   int32_t cnt[2][NQ];    // candidates held, double-buffered by tile parity
   int32_t nvis[NQ];      // keys visible to each query of the group
   int4 wc[2][NQ];        // per-warp pass counts (x..w = warps 0..3), double-buffered by tile parity
-  uint32_t red[24];      // reduction scratch
+  uint32_t red[24];      // reduction scratch (of the second half-group team: red2)
+  uint32_t red2[24];
   int32_t cwc[2][4];     // per-warp counts during compaction (double-buffered)
   int32_t scan[4];       // per-warp totals of a register-resident compaction
   // pruning: folded weights of the kept heads, then Ceff (read as float4)
@@ -423,6 +424,14 @@ __device__ int wg_compact(const uint2* buf, int n, Cut c, bool keep_all, int32_t
 // buffer fits (capacity <= 4,096 entries, i.e. budgets up to 2,048).
 // ------------------------------------------------------------------------
 constexpr int kRegEntries = 32;
+// A selection runs on a team of NW warps (4: a whole epilogue group; 2: half
+// a group, each half selecting for one of the group's two queries) with
+// NW * 32 threads, a histogram of team_bins<NW>() bins in shared memory and
+// radix digits of at most team_digit_bits<NW>() bits.
+template <int NW>
+__host__ __device__ constexpr int team_bins() { return NW == 4 ? kHistBins : kHistBins / 2; }
+template <int NW>
+__host__ __device__ constexpr int team_digit_bits() { return NW == 4 ? kDigitBits : kDigitBits - 1; }
 constexpr int kRegCap = kRegEntries * kBM;
 constexpr int kWarpEntries = kRegEntries * 32;   // entries held by one warp
 
@@ -457,6 +466,7 @@ __device__ __forceinline__ uint32_t rb_field(const RegBuf& b, int r, bool idx_fi
 // Largest and smallest ranked value over the valid entries (only those whose
 // ordered score equals fval when `filt`).  The next pass's barriers order the
 // reuse of `red`.
+template <int NW = 4>
 __device__ inline void rb_maxmin(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t& mx,
                           uint32_t& mn, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
@@ -477,9 +487,14 @@ __device__ inline void rb_maxmin(const RegBuf& b, int n, bool idx_field, bool fi
     red[wq] = mx;
     red[4 + wq] = mn;
   }
-  named_bar(bar_id, kBM);
-  mx = max(max(red[0], red[1]), max(red[2], red[3]));
-  mn = min(min(red[4], red[5]), min(red[6], red[7]));
+  named_bar(bar_id, NW * 32);
+  mx = red[0];
+  mn = red[4];
+#pragma unroll
+  for (int w2 = 1; w2 < NW; ++w2) {
+    mx = max(mx, red[w2]);
+    mn = min(mn, red[4 + w2]);
+  }
 }
 
 struct Digit {
@@ -499,10 +514,12 @@ struct Digit {
 // distinct banks), a suffix scan over the lanes finds the lane holding the
 // rank-th largest, a second scan over that lane's bins finds the digit, and
 // the warp clears the bins.  Two barriers.
+template <int NW>
 __device__ inline Digit rb_find_digit(int nb, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id);
 
 // (entries above `top` are left out: they lie in higher bins of an earlier
 // pass)
+template <int NW = 4>
 __device__ inline Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool filt, uint32_t fval, uint32_t base,
                          int shift, int width, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id,
                          uint32_t top = 0xFFFFFFFFu) {
@@ -517,14 +534,15 @@ __device__ inline Digit rb_pass(const RegBuf& b, int n, bool idx_field, bool fil
                     (static_cast<unsigned long long>(f - base) < span) & (f <= top);
     if (ok) atomicAdd(&hist[(f - base) >> shift], 1u);
   }
-  return rb_find_digit(nb, rank, hist, red, etid, bar_id);
+  return rb_find_digit<NW>(nb, rank, hist, red, etid, bar_id);
 }
 
 // The digit of a filled histogram (2^width = nb bins, counted from the top)
 // that holds the rank-th largest entry; clears the bins.  Two barriers.
+template <int NW>
 __device__ inline Digit rb_find_digit(int nb, uint32_t rank, uint32_t* hist, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
-  named_bar(bar_id, kBM);
+  named_bar(bar_id, NW * 32);
   if (wq == 0) {
     const int per = nb >= 32 ? nb >> 5 : 1;   // bins per lane (a power of two)
     const int owners = nb >= 32 ? 32 : nb;
@@ -557,7 +575,7 @@ __device__ inline Digit rb_find_digit(int nb, uint32_t rank, uint32_t* hist, uin
     __syncwarp();
     for (int i = lane; i < nb; i += 32) hist[i] = 0u;
   }
-  named_bar(bar_id, kBM);
+  named_bar(bar_id, NW * 32);
   return Digit{red[8], red[9], red[10]};
 }
 
@@ -602,19 +620,22 @@ __device__ __forceinline__ void warp_sort64_desc(unsigned long long (&v)[2], int
 // 0 sorts them by (ordered score desc, index asc) and the rank-th of them
 // gives v and the index cut.  red[12] counts the gathered entries (cleared by
 // the caller before its first barrier).
+template <int NW = 4>
 __device__ inline RegCut rb_small_select(const RegBuf& b, int n, uint32_t base, unsigned long long span,
                                          uint32_t rank, uint32_t ksel, uint32_t* hist, uint32_t* red, int etid,
                                          int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
   const int room = rb_room(n, etid);
-  uint2* list = reinterpret_cast<uint2*>(hist + 512);
+  // the upper half of the team's histogram (zero after the passes) holds the
+  // gathered entries: 64 x 8 bytes fit in 256 of its words
+  uint2* list = reinterpret_cast<uint2*>(hist + team_bins<NW>() / 2);
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r) {
     const uint32_t k = b.key[r];
     const bool in = (32 * r < room) & (k >= base) & (static_cast<unsigned long long>(k - base) < span);
     if (in) list[atomicAdd(&red[12], 1u)] = make_uint2(k, b.idx[r]);
   }
-  named_bar(bar_id, kBM);
+  named_bar(bar_id, NW * 32);
   if (wq == 0) {
     const uint32_t m = red[12];
     unsigned long long v[2];
@@ -632,7 +653,7 @@ __device__ inline RegCut rb_small_select(const RegBuf& b, int n, uint32_t base, 
       red[9] = ~static_cast<uint32_t>(w);
     }
   }
-  named_bar(bar_id, kBM);
+  named_bar(bar_id, NW * 32);
   return {red[8], red[9], false, static_cast<int>(ksel)};
 }
 
@@ -640,23 +661,26 @@ __device__ inline RegCut rb_small_select(const RegBuf& b, int n, uint32_t base, 
 // [fmn, fmn + 1024 / scale].  Rounded subtraction, multiplication by a
 // positive scale and truncation are each monotone, so a higher bin holds only
 // strictly higher scores and equal scores share a bin.
+template <int NW = 4>
 __device__ __forceinline__ uint32_t score_bin(uint32_t key, float fmn, float scale) {
-  return min(static_cast<uint32_t>(kHistBins - 1), __float2uint_rz((key_to_float(key) - fmn) * scale));
+  return min(static_cast<uint32_t>(team_bins<NW>() - 1), __float2uint_rz((key_to_float(key) - fmn) * scale));
 }
 
 // First pass over score values: the bin holding the rank-th largest entry.
+template <int NW = 4>
 __device__ inline Digit rb_fpass(const RegBuf& b, int n, float fmn, float scale, uint32_t rank, uint32_t* hist,
                                  uint32_t* red, int etid, int bar_id) {
   const int room = rb_room(n, etid);
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r)
-    if (32 * r < room) atomicAdd(&hist[score_bin(b.key[r], fmn, scale)], 1u);
-  return rb_find_digit(kHistBins, rank, hist, red, etid, bar_id);
+    if (32 * r < room) atomicAdd(&hist[score_bin<NW>(b.key[r], fmn, scale)], 1u);
+  return rb_find_digit<NW>(team_bins<NW>(), rank, hist, red, etid, bar_id);
 }
 
 // Smallest and largest ordered score among the entries of first-pass bin d
 // (the bin is not empty).  One barrier; `red` is reused by the next phase
 // only after its own barrier.
+template <int NW = 4>
 __device__ inline void rb_bin_range(const RegBuf& b, int n, float fmn, float scale, uint32_t d, uint32_t& lo,
                                     uint32_t& hi, uint32_t* red, int etid, int bar_id) {
   const int lane = etid & 31, wq = etid >> 5;
@@ -665,7 +689,7 @@ __device__ inline void rb_bin_range(const RegBuf& b, int n, float fmn, float sca
 #pragma unroll
   for (int r = 0; r < kRegEntries; ++r) {
     const uint32_t k = b.key[r];
-    const bool in = (32 * r < room) & (score_bin(k, fmn, scale) == d);
+    const bool in = (32 * r < room) & (score_bin<NW>(k, fmn, scale) == d);
     mx = max(mx, in ? k : 0u);
     mn = min(mn, in ? k : 0xFFFFFFFFu);
   }
@@ -675,9 +699,14 @@ __device__ inline void rb_bin_range(const RegBuf& b, int n, float fmn, float sca
     red[16 + wq] = mx;
     red[20 + wq] = mn;
   }
-  named_bar(bar_id, kBM);
-  hi = max(max(red[16], red[17]), max(red[18], red[19]));
-  lo = min(min(red[20], red[21]), min(red[22], red[23]));
+  named_bar(bar_id, NW * 32);
+  hi = red[16];
+  lo = red[20];
+#pragma unroll
+  for (int w2 = 1; w2 < NW; ++w2) {
+    hi = max(hi, red[16 + w2]);
+    lo = min(lo, red[20 + w2]);
+  }
 }
 
 // Radix select of the ksel-th largest (ordered score, then lowest index).
@@ -690,39 +719,42 @@ __device__ inline void rb_bin_range(const RegBuf& b, int n, float fmn, float sca
 // bound for a running threshold.  Once the bin holding the ksel-th entry has
 // at most kSmallSel entries, they are sorted in one warp (rb_small_select)
 // instead of further passes.
+template <int NW = 4>
 __device__ inline RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool approx, int room, uint32_t* hist,
                          uint32_t* red, int etid, int bar_id) {
+  constexpr int kBins = team_bins<NW>();
+  constexpr int kBits = team_digit_bits<NW>();
   uint32_t mx, mn;
   // the passes keep the histogram zero between them; the barrier of the
   // max / min below orders this clearing (and of the gather counter) before
   // the first pass
-  for (int i = etid; i < kHistBins; i += kBM) hist[i] = 0u;
+  for (int i = etid; i < kBins; i += NW * 32) hist[i] = 0u;
   if (etid == 0) red[12] = 0u;
-  rb_maxmin(b, n, false, false, 0u, mx, mn, red, etid, bar_id);
+  rb_maxmin<NW>(b, n, false, false, 0u, mx, mn, red, etid, bar_id);
   uint32_t base = mn, above = 0u, cnt = static_cast<uint32_t>(n), rank = ksel;
   if (mx != mn) {
     const float fmn = key_to_float(mn);
-    float scale = static_cast<float>(kHistBins) / (key_to_float(mx) - fmn);
+    float scale = static_cast<float>(kBins) / (key_to_float(mx) - fmn);
     if (!(scale < 1.0e30f)) scale = 0.f;  // a span too narrow for float bins: one bin, passes below
-    const Digit d0 = rb_fpass(b, n, fmn, scale, rank, hist, red, etid, bar_id);
+    const Digit d0 = rb_fpass<NW>(b, n, fmn, scale, rank, hist, red, etid, bar_id);
     above += d0.above;
     rank -= d0.above;
     cnt = d0.cnt;
     uint32_t lo, hi;
-    rb_bin_range(b, n, fmn, scale, d0.d, lo, hi, red, etid, bar_id);
+    rb_bin_range<NW>(b, n, fmn, scale, d0.d, lo, hi, red, etid, bar_id);
     // every entry of a higher bin scores above hi, every entry of a lower
     // one below lo: [lo, hi] holds exactly the bin's entries
     if (approx && static_cast<int>(above + cnt) <= room) return {lo, 0u, true, static_cast<int>(above + cnt)};
     if (cnt <= static_cast<uint32_t>(kSmallSel))
-      return rb_small_select(b, n, lo, static_cast<unsigned long long>(hi - lo) + 1ull, rank, ksel, hist, red,
-                             etid, bar_id);
+      return rb_small_select<NW>(b, n, lo, static_cast<unsigned long long>(hi - lo) + 1ull, rank, ksel, hist, red,
+                                 etid, bar_id);
     base = lo;
     if (hi != lo) {
       int shift = 32 - __clz(hi - lo);  // bits of the bin's span of ordered scores
       while (shift > 0) {
-        const int width = shift < kDigitBits ? shift : kDigitBits;
+        const int width = shift < kBits ? shift : kBits;
         shift -= width;
-        const Digit dg = rb_pass(b, n, false, false, 0u, base, shift, width, rank, hist, red, etid, bar_id, hi);
+        const Digit dg = rb_pass<NW>(b, n, false, false, 0u, base, shift, width, rank, hist, red, etid, bar_id, hi);
         base += dg.d << shift;
         above += dg.above;
         rank -= dg.above;
@@ -730,8 +762,8 @@ __device__ inline RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool appr
         if (cnt <= static_cast<uint32_t>(kSmallSel)) {
           const unsigned long long digit_span = 1ull << shift;
           const unsigned long long to_hi = static_cast<unsigned long long>(hi - base) + 1ull;
-          return rb_small_select(b, n, base, digit_span < to_hi ? digit_span : to_hi, rank, ksel, hist, red,
-                                 etid, bar_id);
+          return rb_small_select<NW>(b, n, base, digit_span < to_hi ? digit_span : to_hi, rank, ksel, hist, red,
+                                     etid, bar_id);
         }
       }
     }
@@ -740,18 +772,18 @@ __device__ inline RegCut rb_cut(const RegBuf& b, int n, uint32_t ksel, bool appr
   // entries tied at v make the cut
   if (rank >= cnt) return {base, 0xFFFFFFFFu, false, static_cast<int>(above + cnt)};
   if (cnt <= static_cast<uint32_t>(kSmallSel))
-    return rb_small_select(b, n, base, 1ull, rank, ksel, hist, red, etid, bar_id);
+    return rb_small_select<NW>(b, n, base, 1ull, rank, ksel, hist, red, etid, bar_id);
   // many ties at v: the rank-th largest ~index among them, by the same passes
   const uint32_t v = base;
   uint32_t imx, imn;
-  rb_maxmin(b, n, true, true, v, imx, imn, red, etid, bar_id);
+  rb_maxmin<NW>(b, n, true, true, v, imx, imn, red, etid, bar_id);
   uint32_t ibase = imn;
   if (imx != imn) {
     int shift = 32 - __clz(imx - imn);
     while (shift > 0) {
-      const int width = shift < kDigitBits ? shift : kDigitBits;
+      const int width = shift < kBits ? shift : kBits;
       shift -= width;
-      const Digit dg = rb_pass(b, n, true, true, v, ibase, shift, width, rank, hist, red, etid, bar_id);
+      const Digit dg = rb_pass<NW>(b, n, true, true, v, ibase, shift, width, rank, hist, red, etid, bar_id);
       ibase += dg.d << shift;
       rank -= dg.above;
     }
@@ -1423,8 +1455,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         // cap - kBM >= cut_min) and those of the joining groups that are well
         // on their way
         const int cut_min = kRounds ? (p.cap + p.ksel) / 2 : p.cap - kBM;
+        // Two queries per group and both buffers within two warps' registers
+        // (2,048 entries): warps 0-1 and 2-3 select for query 0 and query 1
+        // at once, each on half of the group's histogram, instead of the
+        // whole group selecting for one query after the other.
+        bool halves_done = false;
+        if constexpr (kDefer && NQW == 2) {
+          const int n0 = st->cnt[par][0], n1 = st->cnt[par][1];
+          if (fin && n0 <= kRegCap / 2 && n1 <= kRegCap / 2) {
+            const int h = wq >> 1;
+            const int qi = h;
+            const int tid = etid - h * 64;
+            const int n = h ? n1 : n0;
+            const int64_t t = tq0 + qi;
+            uint4 job = make_uint4(static_cast<uint32_t>(n), 0u, 0xFFFFFFFFu, t < p.S ? kJobAll : kJobSkip);
+            if (t < p.S && n > p.ksel) {
+              RegBuf rb;
+              rb_load(rb, cand + qi * static_cast<size_t>(p.cap), n, tid);
+              const RegCut c = rb_cut<2>(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist + h * (kHistBins / 2),
+                                         h ? st->red2 : st->red, tid, 5 + 2 * eg + h);
+              job = make_uint4(static_cast<uint32_t>(n), c.v, c.icut, kJobCut);
+            }
+            if (tid == 0) bars->jobs[set][eg][qi] = job;
+            named_bar(bar_id, kBM);
+            halves_done = true;
+          }
+        }
 #pragma unroll 1
-        for (int qi = 0; qi < NQW; ++qi) {
+        for (int qi = 0; qi < (halves_done ? 0 : NQW); ++qi) {
           const int n = st->cnt[par][qi];
           const int64_t t = tq0 + qi;
           if (kDefer && fin && etid == 0 && t >= p.S) bars->jobs[set][eg][qi] = make_uint4(0u, 0u, 0u, kJobSkip);
