@@ -160,6 +160,26 @@ def flops_per_pair(wl):
     return 2.0 * wl.H * wl.D
 
 
+def hbm_summary(wl, rows, kern_ms, peak_gbs):
+    """Algorithmic HBM traffic of one indexer call over `rows` query rows (read
+    q, k, w, the scales and pool coefficients once, write idx and len once),
+    its rate over the call's device time, and the [rows, keys] FP32 score
+    tensor a materialising indexer would write instead."""
+    elem = 1 if wl.dtype == "fp8" else 2
+    pooled = wl.visibility == W.POOLED
+    n_keys = wl.T // wl.ratio if pooled else wl.T        # scored keys (pools for POOLED)
+    width = wl.K + wl.ratio - 1 if pooled else wl.K
+    read = rows * wl.H * wl.D * elem + wl.T * wl.D * elem + rows * wl.H * 4
+    if wl.dtype == "fp8":
+        read += rows * wl.H * 4 + wl.T * 4
+    if pooled:
+        read += wl.ratio * wl.D * 2
+    write = rows * width * 4 + rows * 4
+    achieved = (read + write) / (kern_ms * 1e-3) / 1e9
+    return {"algorithmic_bytes": read + write, "achieved_gbs": achieved, "peak_gbs": peak_gbs,
+            "frac": achieved / peak_gbs, "materialised_scores_gib": rows * n_keys * 4 / 2**30}
+
+
 def rank_part(wl, rank, world, scaling):
     """(workload whose inputs this rank draws, first row, end row) of this
     rank's share.  Strong scaling: every rank draws the whole workload (the
@@ -384,6 +404,7 @@ def measure(wl, inp, r0, r1, steps, warmup, dev, world, local, with_e2e=False, e
                      "peak_source": f"{pk['source']} bf16 burst" + (" x2 for fp8 (nominal ratio)" if wl.dtype == "fp8" else ""),
                      "flops_per_pair": flops_per_pair(wl)},
         "clocks": clk.summary(), "device_status": status,
+        "hbm": hbm_summary(wl, r1 - r0, kern_ms, pk["hbm"]),
     }
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     splits = planned_splits(wl, S, wl.q_pos0 + r0, sms)
@@ -564,6 +585,7 @@ def main():
             "tensor_peak_frac": res["tensor_peak_frac"],
             "peak_hbm_gb": res["peak_hbm_gb"],
             "roofline": roof,
+            "hbm": res["hbm"],
             "clocks": res["clocks"],
             "e2e": res.get("e2e"),
             "gpu_launches": res["launches_per_step"] * args.steps,

@@ -4,7 +4,9 @@
 // indexer_read_status, which says so).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "hwr_indexer.h"
 #include "internal.h"
@@ -359,6 +361,7 @@ indexer_status run_topk(const indexer_problem* p, const void* q, const void* k, 
   sp.split_rth = split_rth;
   sp.seed_thr = nullptr;
   sp.test_wait_ns = (p->flags & INDEXER_FLAG_TEST_WAIT_TIMEOUT) ? 1000000 : 0;
+  sp.seg = nullptr;
   if (seeds) {
     WitnessParams wp;
     wp.S = p->S;
@@ -727,6 +730,176 @@ indexer_status doc_part(const indexer_problem* p, const int64_t* b, int32_t d, D
   return INDEXER_OK;
 }
 
+// Packed documents of token or compressed keys, without the pruning
+// certificate and the test hook, run as one launch of the segmented kernel
+// (every document's query blocks in one table) when the batch has more query
+// blocks than half the SMs but its documents average fewer than two blocks
+// per SM.  Fewer blocks in all (a few queries at the end of long documents)
+// keep one launch per document, which can split each block's keys over
+// several CTAs; long documents keep it too, since each launch then fills
+// the GPU (measured: 64 documents of 4,096 tokens 19.9 ms in 64 launches,
+// 21.9 ms in one; 1,024 of 256 tokens 25.2 ms against 6.6 ms).
+indexer_status docs_fold(const indexer_problem* p, const int64_t* b, int32_t n_docs, bool* fold);
+
+// The segmented launch of a packed batch: the whole problem's plan with one
+// range per block and a grid over the table's blocks, the block table sorted
+// by key tiles, lightest first (the kernel deals blocks out heaviest first),
+// and the workspace (status block, candidate buffers, table).
+struct SegPlan {
+  Plan pl;
+  std::vector<SegBlock> blocks;
+  size_t cand_off, table_off, ws_bytes;
+};
+
+indexer_status seg_plan(const indexer_problem* p, const int64_t* b, int32_t n_docs, SegPlan* sp) {
+  indexer_status st = make_plan(p, true, &sp->pl);
+  if (st != INDEXER_OK) return st;
+  Plan& pl = sp->pl;
+  DeviceInfo di;
+  st = device_info(&di);
+  if (st != INDEXER_OK) return st;
+  const int64_t qb = pl.var.queries_per_block;
+  const int64_t ratio = pl.ranged ? p->ratio : 1;
+  sp->blocks.clear();
+  for (int32_t d = 0; d < n_docs; ++d) {
+    DocPart part;
+    bool empty = false;
+    st = doc_part(p, b, d, &part, &empty);
+    if (st != INDEXER_OK) return st;
+    if (empty) continue;
+    if (part.sub.T > INT32_MAX || part.key0 > INT32_MAX) return INDEXER_EUNSUPPORTED;
+    for (int64_t r = 0; r < part.sub.S; r += qb) {
+      SegBlock blk;
+      blk.row0 = part.r0 + r;
+      blk.pos0 = part.sub.q_pos0 + r;
+      blk.key0 = part.key0;
+      blk.rows = static_cast<int32_t>(part.sub.S - r < qb ? part.sub.S - r : qb);
+      blk.n_keys = static_cast<int32_t>(part.sub.T);
+      sp->blocks.push_back(blk);
+    }
+  }
+  if (sp->blocks.size() > static_cast<size_t>(INT32_MAX)) return INDEXER_EUNSUPPORTED;
+  auto tiles = [&](const SegBlock& blk) {
+    const int64_t g = blk.pos0 + blk.rows - 1;
+    int64_t n = pl.ranged ? (g + 1) / ratio : g + 1;
+    if (n > blk.n_keys) n = blk.n_keys;
+    return (n + 127) / 128;
+  };
+  std::stable_sort(sp->blocks.begin(), sp->blocks.end(),
+                   [&](const SegBlock& x, const SegBlock& y) { return tiles(x) < tiles(y); });
+  const int64_t nb = static_cast<int64_t>(sp->blocks.size());
+  pl.n_blocks = static_cast<int32_t>(nb);
+  pl.splits = 1;
+  pl.split_bytes = pl.gather_bytes = pl.split_cnt_bytes = 0;
+  pl.gather_stride = 0;
+  pl.grid = static_cast<int32_t>(nb < di.sms ? nb : di.sms);
+  pl.cand_bytes = static_cast<size_t>(pl.grid) * kCandSets * pl.var.groups * pl.var.queries_per_wg *
+                  static_cast<size_t>(pl.cap) * sizeof(uint2);
+  sp->cand_off = kStatusBytes;
+  sp->table_off = sp->cand_off + align256(pl.cand_bytes);
+  sp->ws_bytes = sp->table_off + align256(sp->blocks.size() * sizeof(SegBlock));
+  return INDEXER_OK;
+}
+
+// The segmented launch itself: the block table copied into the workspace
+// (a small copy from host memory, staged by the driver), then one launch
+// over every document's blocks.  Output indices carry each document's key
+// offset, so no separate shift pass runs.
+indexer_status run_seg(const indexer_problem* p, const int64_t* b, int32_t n_docs, const void* q, const void* k,
+                       const float* w, const float* q_scale, const float* k_scale, int32_t* out_idx,
+                       int32_t* out_len, float* out_score, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  SegPlan sp;
+  indexer_status st = seg_plan(p, b, n_docs, &sp);
+  if (st != INDEXER_OK) return st;
+  const Plan& pl = sp.pl;
+  DeviceInfo di;
+  st = device_info(&di);
+  if (st != INDEXER_OK) return st;
+  if (!di.sm100) return INDEXER_EDEVICE;
+  if (!pl.var.fn_seg) return INDEXER_EUNSUPPORTED;
+  const bool fp8 = p->dtype == INDEXER_FP8_E4M3;
+  if (!k || !aligned(k, 16) || (q && !aligned(q, 16))) return INDEXER_EINVAL;
+  if (workspace_bytes < sp.ws_bytes) return INDEXER_EWORKSPACE;
+  if (!get_encoder()) return INDEXER_ECUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, 32, stream) != cudaSuccess) return INDEXER_ECUDA;
+  if (p->S == 0 || sp.blocks.empty()) return INDEXER_OK;
+  SegBlock* table = reinterpret_cast<SegBlock*>(ws + sp.table_off);
+  if (cudaMemcpyAsync(table, sp.blocks.data(), sp.blocks.size() * sizeof(SegBlock), cudaMemcpyHostToDevice,
+                      stream) != cudaSuccess)
+    return INDEXER_ECUDA;
+  CUtensorMap tm_q, tm_k;
+  if (!encode_2d(&tm_q, q, fp8, p->S * p->H, p->D, pl.var.q_box_rows)) return INDEXER_ECUDA;
+  if (!encode_2d(&tm_k, k, fp8, pl.n_keys > 0 ? pl.n_keys : 1, p->D, 128)) return INDEXER_ECUDA;
+  ScoreParams prm{};
+  prm.S = p->S;
+  prm.n_keys = pl.n_keys;
+  prm.q_pos0 = p->q_pos0;
+  prm.ranged = pl.ranged;
+  prm.ratio = pl.ranged ? p->ratio : 1;
+  prm.out_ratio = 1;
+  prm.out_ratio_inv = 0u;
+  prm.ksel = pl.ksel;
+  prm.width = pl.width;
+  prm.n_blocks = pl.n_blocks;
+  prm.cap = pl.cap;
+  prm.w = w;
+  prm.q_scale = q_scale;
+  prm.k_scale = k_scale;
+  prm.out_idx = out_idx;
+  prm.out_len = out_len;
+  prm.out_score = out_score;
+  prm.cand = reinterpret_cast<uint2*>(ws + sp.cand_off);
+  prm.status = reinterpret_cast<uint32_t*>(ws);
+  prm.prune = 0;
+  prm.pq = nullptr;
+  prm.knorm = nullptr;
+  prm.counters = reinterpret_cast<unsigned long long*>(ws + 8);
+  prm.splits = 1;
+  prm.split_buf = nullptr;
+  prm.split_cnt = nullptr;
+  prm.split_kth = nullptr;
+  prm.split_rth = nullptr;
+  prm.seed_thr = nullptr;
+  prm.test_wait_ns = 0;
+  prm.seg = table;
+  if (cudaFuncSetAttribute(pl.var.fn_seg, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.var.smem_bytes) !=
+      cudaSuccess)
+    return INDEXER_ECUDA;
+  void* args[] = {&tm_q, &tm_k, &prm};
+  if (cudaLaunchKernel(pl.var.fn_seg, dim3(pl.grid), dim3(pl.var.threads), args, pl.var.smem_bytes, stream) !=
+      cudaSuccess)
+    return INDEXER_ECUDA;
+  return INDEXER_OK;
+}
+
+indexer_status docs_fold(const indexer_problem* p, const int64_t* b, int32_t n_docs, bool* fold) {
+  *fold = false;
+  if (p->visibility == INDEXER_VIS_POOLED || (p->flags & (INDEXER_FLAG_PRUNE | INDEXER_FLAG_TEST_WAIT_TIMEOUT)) != 0)
+    return INDEXER_OK;
+  Plan pl;
+  indexer_status st = make_plan(p, false, &pl);
+  if (st != INDEXER_OK) return st;
+  DeviceInfo di;
+  st = device_info(&di);
+  if (st != INDEXER_OK) return st;
+  const int64_t qb = pl.var.queries_per_block;
+  int64_t nb = 0, docs = 0;
+  for (int32_t d = 0; d < n_docs; ++d) {
+    DocPart part;
+    bool empty = false;
+    st = doc_part(p, b, d, &part, &empty);
+    if (st != INDEXER_OK) return st;
+    if (!empty) {
+      nb += (part.sub.S + qb - 1) / qb;
+      ++docs;
+    }
+  }
+  *fold = nb * 2 > di.sms && nb < docs * 2 * di.sms;
+  return INDEXER_OK;
+}
+
 // Bounds must rise strictly, cover every query position, stay within the
 // keys, and (compressed keys) start documents on a whole compressed key.
 indexer_status check_docs(const indexer_problem* p, const int64_t* b, int32_t n_docs) {
@@ -755,6 +928,16 @@ indexer_status indexer_docs_workspace_bytes(const indexer_problem* p, const int6
   indexer_status st = check_docs(p, doc_bounds, n_docs);
   if (st != INDEXER_OK) return st;
   if (!bytes) return INDEXER_EINVAL;
+  bool fold = false;
+  st = hwr::docs_fold(p, doc_bounds, n_docs, &fold);
+  if (st != INDEXER_OK) return st;
+  if (fold) {
+    hwr::SegPlan sp;
+    st = hwr::seg_plan(p, doc_bounds, n_docs, &sp);
+    if (st != INDEXER_OK) return st;
+    *bytes = sp.ws_bytes;
+    return INDEXER_OK;
+  }
   size_t most = 0;
   for (int32_t d = 0; d < n_docs; ++d) {
     DocPart part;
@@ -904,6 +1087,12 @@ indexer_status indexer_topk_docs(const indexer_problem* p, const void* q, const 
   if (st != INDEXER_OK) return st;
   if (!workspace || !aligned(workspace, 256)) return INDEXER_EWORKSPACE;
   if (workspace_bytes < need) return INDEXER_EWORKSPACE;
+  bool fold = false;
+  st = hwr::docs_fold(p, doc_bounds, n_docs, &fold);
+  if (st != INDEXER_OK) return st;
+  if (fold)
+    return hwr::run_seg(p, doc_bounds, n_docs, q, k, w, q_scale, k_scale, out_idx, out_len, out_score, workspace,
+                        workspace_bytes, static_cast<cudaStream_t>(stream));
   const bool fp8 = p->dtype == INDEXER_FP8_E4M3;
   const size_t elem = fp8 ? 1 : 2;
   int32_t width = 0;

@@ -20,6 +20,18 @@ constexpr int kCandSets = 3;
 // Heads the pruning certificate keeps exactly (the first kPruneR of each query).
 constexpr int kPruneR = 16;
 
+// One query block of a launch over several documents (the segmented kernel):
+// its rows in the batch, the visibility position of its first row within its
+// document, and the document's keys.  Output indices are shifted by key0 (the
+// document's first key row), which numbers them within the whole batch.
+struct SegBlock {
+  int64_t row0;    // first query row of the block
+  int64_t pos0;    // position of row0 within its document (visibility)
+  int64_t key0;    // the document's first key row
+  int32_t rows;    // query rows of the block (at most the block size)
+  int32_t n_keys;  // the document's keys (tokens or compressed keys)
+};
+
 // Arguments of the scoring + top-K kernel (one launch per indexer call).
 struct ScoreParams {
   int64_t S;          // query rows
@@ -53,12 +65,14 @@ struct ScoreParams {
                          // (0 when it has fewer than r)
   const uint32_t* seed_thr;  // [S] ordered-score threshold every query starts from, or null (0 for all)
   int64_t test_wait_ns;  // > 0: test hook, the MMA issuer waits this long on a barrier nothing arrives at
+  const SegBlock* seg;   // segmented kernel: [n_blocks] query blocks, lightest first; else null
 };
 
 // Per-variant launch facts, filled by the kernel's translation unit.
 struct ScoreVariant {
   const void* fn;         // kernel function
   const void* fn_split;   // the same with key ranges split across CTAs (ScoreParams::splits > 1)
+  const void* fn_seg;     // the same over a table of query blocks of several documents (ScoreParams::seg)
   int queries_per_block;  // QB
   int queries_per_wg;     // queries owned by one epilogue warpgroup
   int groups;             // epilogue warpgroups per CTA

@@ -165,6 +165,31 @@ __device__ __forceinline__ int32_t n_visible(const ScoreParams& p, int64_t g) {
   const int64_t n = p.ranged ? (g + 1) / p.ratio : g + 1;
   return static_cast<int32_t>(n < p.n_keys ? n : p.n_keys);
 }
+// the same against a document's own key count
+__device__ __forceinline__ int32_t n_visible_in(const ScoreParams& p, int64_t g, int32_t n_keys) {
+  const int64_t n = p.ranged ? (g + 1) / p.ratio : g + 1;
+  return static_cast<int32_t>(n < n_keys ? n : n_keys);
+}
+
+// Where query block b sits: its first row, the visibility position of that
+// row, the first key row of its keys, its row count and its key count.  A
+// single problem's blocks are QB consecutive rows over all keys; the
+// segmented kernel reads them from its block table.
+struct BlockGeom {
+  int64_t row0, pos0, key0;
+  int32_t rows, n_keys;
+};
+template <int QB, bool SEG>
+__device__ __forceinline__ BlockGeom geom_of(const ScoreParams& p, int b) {
+  if constexpr (SEG) {
+    const SegBlock sb = p.seg[b];
+    return {sb.row0, sb.pos0, sb.key0, sb.rows, sb.n_keys};
+  } else {
+    const int64_t row0 = static_cast<int64_t>(b) * QB;
+    const int64_t left = p.S - row0;
+    return {row0, p.q_pos0 + row0, 0, static_cast<int32_t>(left < QB ? left : QB), static_cast<int32_t>(p.n_keys)};
+  }
+}
 
 // Heaviest query blocks first (they see the most keys), dealt to the CTAs in
 // a snake order so that per-CTA work evens out.  -1 once this CTA is done.
@@ -173,11 +198,10 @@ __device__ __forceinline__ int block_of(int round, int cta, int grid, int n_bloc
   return item < n_blocks ? n_blocks - 1 - item : -1;
 }
 
-template <int QB>
+template <int QB, bool SEG>
 __device__ __forceinline__ int tiles_of_block(const ScoreParams& p, int b) {
-  int64_t t_last = static_cast<int64_t>(b + 1) * QB - 1;
-  if (t_last >= p.S) t_last = p.S - 1;
-  const int32_t n = n_visible(p, p.q_pos0 + t_last);
+  const BlockGeom g = geom_of<QB, SEG>(p, b);
+  const int32_t n = n_visible_in(p, g.pos0 + g.rows - 1, g.n_keys);
   return (n + kBM - 1) / kBM;
 }
 
@@ -188,17 +212,17 @@ __device__ __forceinline__ int tiles_of_block(const ScoreParams& p, int b) {
 struct Item {
   int b, j0, j1, sp;
 };
-template <int QB, bool SPLIT>
+template <int QB, bool SPLIT, bool SEG = false>
 __device__ __forceinline__ Item item_of(const ScoreParams& p, int round, int cta, int grid) {
   if constexpr (!SPLIT) {
     const int b = block_of(round, cta, grid, p.n_blocks);
-    return {b, 0, b < 0 ? 0 : tiles_of_block<QB>(p, b), 0};
+    return {b, 0, b < 0 ? 0 : tiles_of_block<QB, SEG>(p, b), 0};
   }
   const int it = block_of(round, cta, grid, p.n_blocks * p.splits);
   if (it < 0) return {-1, 0, 0, 0};
   const int b = it / p.splits;
   const int sp = it - b * p.splits;
-  const int nt = tiles_of_block<QB>(p, b);
+  const int nt = tiles_of_block<QB, false>(p, b);
   const int per = (nt + p.splits - 1) / p.splits;
   const int j0 = min(sp * per, nt);
   return {b, j0, min(j0 + per, nt), sp};
@@ -878,9 +902,11 @@ __device__ __forceinline__ void emit_expanded(bool keep, int pos, uint32_t key, 
 // incomplete pool's positions appended ("Module 06 — DSA & KPool", §2), then
 // -1 padding and the valid length.  Entries are read two warp-steps at a time
 // so that two loads are in flight.  `stage` is 64 words of this warp's
-// shared memory.
-__device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScoreParams& p, int64_t t,
-                                      uint32_t* stage, int lane) {
+// shared memory.  g is the row's visibility position, n_keys its keys, and
+// `shift` is added to every key index (a document's first key row in a
+// segmented launch, else 0; pooled rows always have 0).
+__device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScoreParams& p, int64_t t, int64_t g,
+                                      int32_t n_keys, int32_t shift, uint32_t* stage, int lane) {
   const int n = static_cast<int>(job.x);
   const bool all = job.w == kJobAll;
   const uint32_t v = all ? 0u : job.y;
@@ -905,7 +931,7 @@ __device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScorePa
       const int pos = kept + __popc(bal & lt);
       if (m == 1) {
         if (keep) {
-          __stcs(&orow[pos], static_cast<int32_t>(e[u].y));
+          __stcs(&orow[pos], static_cast<int32_t>(e[u].y) + shift);
           if (srow) srow[pos] = key_to_float(e[u].x);
         }
       } else if (bal != 0u) {
@@ -916,7 +942,6 @@ __device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScorePa
   }
   int len = kept * m;
   if (m > 1) {
-    const int64_t g = p.q_pos0 + t;
     const int tail = static_cast<int>((g + 1) % m);
     const int64_t first = g + 1 - tail;
     for (int i = lane; i < tail; i += 32) {
@@ -932,14 +957,14 @@ __device__ inline void warp_write_row(const uint2* buf, uint4 job, const ScorePa
   if (lane == 0) {
     p.out_len[t] = len;
     // with a seed threshold at least min(K, visible) keys must pass it
-    if (p.seed_thr != nullptr && kept < min(p.ksel, n_visible(p, p.q_pos0 + t))) atomicOr(p.status, kStatusWitness);
+    if (p.seed_thr != nullptr && kept < min(p.ksel, n_visible_in(p, g, n_keys))) atomicOr(p.status, kStatusWitness);
   }
 }
 
 // ------------------------------------------------------------------------
 // The kernel.
 // ------------------------------------------------------------------------
-template <int H, int D, bool FP8, bool PRUNE, bool SPLIT>
+template <int H, int D, bool FP8, bool PRUNE, bool SPLIT, bool SEG = false>
 __global__ void __launch_bounds__(kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const ScoreParams p) {
@@ -1016,7 +1041,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and q blocks; after an abort the last ones may still be landing
       uint32_t n_kloads = 0, n_qloads = 0;
       for (int r = 0; ok; ++r) {
-        const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+        const Item it = item_of<QB, SPLIT, SEG>(p, r, blockIdx.x, gridDim.x);
         const int b = it.b;
         if (b < 0) break;
         if (it.j1 == it.j0) continue;
@@ -1027,10 +1052,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         first = false;
         ++n_qloads;
+        // the block's q rows (a segmented launch: rows of one document, the
+        // box's rows past them are scored and never used) and its keys
+        const BlockGeom bg = geom_of<QB, SEG>(p, b);
+        const int32_t q_row = static_cast<int32_t>(bg.row0 * H);
+        const int32_t k_row0 = static_cast<int32_t>(bg.key0);
         mbar_arrive_expect_tx(&bars->qfull, C::Q_BYTES);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_2d_hint(smem + C::OFF_Q + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS, b * QB * H, &bars->qfull, pol_q);
+          tma_load_2d_hint(smem + C::OFF_Q + bx * BN * 128, &tm_q, bx * C::BOX_ELEMS, q_row, &bars->qfull, pol_q);
         for (int j = it.j0; j < it.j1; ++j) {
           ok = mbar_wait(&bars->kempty[stage], kph ^ 1u, abort_flag, kWaitLimitNs);
           if (!ok) break;
@@ -1039,7 +1069,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int bx = 0; bx < C::NBOX; ++bx)
             tma_load_2d_hint(smem + C::OFF_K + stage * C::K_STAGE_BYTES + bx * kBM * 128, &tm_k, bx * C::BOX_ELEMS,
-                             j * kBM, &bars->kfull[stage], pol_k);
+                             k_row0 + j * kBM, &bars->kfull[stage], pol_k);
           if (++stage == STAGES) {
             stage = 0;
             kph ^= 1u;
@@ -1064,7 +1094,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t tcount = 0;  // tiles issued so far; tile n goes to accumulator n & 1
       bool ok = true;
       for (int r = 0; ok; ++r) {
-        const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+        const Item it = item_of<QB, SPLIT, SEG>(p, r, blockIdx.x, gridDim.x);
         if (it.b < 0) break;
         const int nt = it.j1 - it.j0;
         if (nt == 0) continue;
@@ -1128,8 +1158,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // queries' candidate buffers (one of two sets) with their final cuts.
     const int ww = warp - 2;
     for (int r = 0;; ++r) {
-      const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+      const Item it = item_of<QB, SPLIT, SEG>(p, r, blockIdx.x, gridDim.x);
       if (it.b < 0) break;
+      const BlockGeom bg = geom_of<QB, SEG>(p, it.b);
       const int set = r % kSets;
       bool ok = mbar_wait(&bars->fin_full[set], static_cast<uint32_t>(r / kSets) & 1u, abort_flag, kWaitLimitNs);
       if (!__any_sync(kFullMask, ok)) {
@@ -1143,11 +1174,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = jb / NQW, qi = jb - g * NQW;
         const uint4 job = bars->jobs[set][g][qi];
         if (job.w == kJobSkip) continue;
-        const int64_t t = static_cast<int64_t>(it.b) * QB + g * NQW + qi;
+        const int local = g * NQW + qi;  // row within the block
         const uint2* buf = p.cand + ((static_cast<size_t>(blockIdx.x) * kSets + set) * kEpiGroups + g) * NQW *
                                         static_cast<size_t>(p.cap) +
                            qi * static_cast<size_t>(p.cap);
-        warp_write_row(buf, job, p, t, bars->fstage[ww], lane);
+        warp_write_row(buf, job, p, bg.row0 + local, bg.pos0 + local, bg.n_keys, static_cast<int32_t>(bg.key0),
+                       bars->fstage[ww], lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->fin_free[set]);
@@ -1204,11 +1236,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool failed = false;
     unsigned long long n_screened = 0ull, n_bounded = 0ull, n_skipped = 0ull;  // pruning counters (lane 0)
     for (int r = 0; !failed; ++r) {
-      const Item it = item_of<QB, SPLIT>(p, r, blockIdx.x, gridDim.x);
+      const Item it = item_of<QB, SPLIT, SEG>(p, r, blockIdx.x, gridDim.x);
       const int b = it.b;
       if (b < 0) break;
       const int nt = it.j1;
-      const int64_t tq0 = static_cast<int64_t>(b) * QB + eg * NQW;
+      // the block's rows [row0, t_end), their visibility origin and keys
+      const BlockGeom bg = geom_of<QB, SEG>(p, b);
+      const int64_t tq0 = bg.row0 + eg * NQW;
+      const int64_t t_end = SEG ? bg.row0 + bg.rows : p.S;
+      const int64_t pos_shift = SEG ? bg.pos0 - bg.row0 : p.q_pos0;  // visibility position = t + pos_shift
+      const int64_t kcap = SEG ? bg.n_keys : p.n_keys;
+      const float* ksc = FP8 ? p.k_scale + (SEG ? bg.key0 : 0) : nullptr;
+      const int32_t out_shift = SEG ? static_cast<int32_t>(bg.key0) : 0;
       const int set = r % kSets;  // candidate-buffer set of this block
       uint2* cand = p.cand + ((static_cast<size_t>(blockIdx.x) * kSets + set) * kEpiGroups + eg) * NQW *
                                  static_cast<size_t>(p.cap);
@@ -1227,7 +1266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = etid; i < C::CW; i += kBM) {
         const int64_t t = tq0 + i / H;
         float v = 0.f;
-        if (t < p.S) {
+        if (t < t_end) {
           v = p.w[t * H + (i % H)];
           if constexpr (FP8) v *= p.q_scale[t * H + (i % H)];
         }
@@ -1237,17 +1276,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = etid; i < NQW * (kPruneR + 2); i += kBM) {
           const int qi = i / (kPruneR + 2), c = i % (kPruneR + 2);
           const int64_t t = tq0 + qi;
-          const float v = t < p.S ? p.pq[t * (kPruneR + 2) + c] : 0.f;
+          const float v = t < t_end ? p.pq[t * (kPruneR + 2) + c] : 0.f;
           st->pq[qi][c] = c < kPruneR ? 0.5f * v : v;  // kept-head weights halved, as for relu2
         }
       }
       if (kRounds && etid == 0) *seen = *cut_round;
       if (etid < NQW) {
         const int64_t t = tq0 + etid;
-        st->nvis[etid] = t < p.S ? n_visible(p, p.q_pos0 + t) : 0;
+        st->nvis[etid] = t < t_end ? n_visible_in(p, t + pos_shift, static_cast<int32_t>(kcap)) : 0;
         st->cnt[par][etid] = 0;
         // a seed threshold, when given, is a lower bound of the K-th score
-        st->thr[etid] = (p.seed_thr != nullptr && t < p.S) ? p.seed_thr[t] : 0u;
+        st->thr[etid] = (p.seed_thr != nullptr && t < t_end) ? p.seed_thr[t] : 0u;
       }
       named_bar(bar_id, kBM);
 
@@ -1294,8 +1333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float ks_next = 1.f, kn_next = 0.f;
         {
           const int32_t key = j * kBM + etid;
-          if constexpr (FP8) ks_next = (j < nt && key < p.n_keys) ? p.k_scale[key] : 0.f;
-          if constexpr (PRUNE) kn_next = (j < nt && key < p.n_keys) ? p.knorm[key] : 0.f;
+          if constexpr (FP8) ks_next = (j < nt && key < kcap) ? ksc[key] : 0.f;
+          if constexpr (PRUNE) kn_next = (j < nt && key < kcap) ? p.knorm[key] : 0.f;
         }
         for (; j < nt; ++j) {
           const int a = static_cast<int>(tcount % C::NACC);
@@ -1304,8 +1343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float ks = ks_next, kn = kn_next;
           if (FP8 || PRUNE) {
             const int32_t key1 = key + kBM;
-            const bool more = j + 1 < nt && key1 < p.n_keys;
-            if constexpr (FP8) ks_next = more ? p.k_scale[key1] : 0.f;
+            const bool more = j + 1 < nt && key1 < kcap;
+            if constexpr (FP8) ks_next = more ? ksc[key1] : 0.f;
             if constexpr (PRUNE) kn_next = more ? p.knorm[key1] : 0.f;
           }
           // every lane polls (no divergent branch around the wait); the phase
@@ -1468,8 +1507,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int tid = etid - h * 64;
             const int n = h ? n1 : n0;
             const int64_t t = tq0 + qi;
-            uint4 job = make_uint4(static_cast<uint32_t>(n), 0u, 0xFFFFFFFFu, t < p.S ? kJobAll : kJobSkip);
-            if (t < p.S && n > p.ksel) {
+            uint4 job = make_uint4(static_cast<uint32_t>(n), 0u, 0xFFFFFFFFu, t < t_end ? kJobAll : kJobSkip);
+            if (t < t_end && n > p.ksel) {
               RegBuf rb;
               rb_load(rb, cand + qi * static_cast<size_t>(p.cap), n, tid);
               const RegCut c = rb_cut<2>(rb, n, static_cast<uint32_t>(p.ksel), false, 0, hist + h * (kHistBins / 2),
@@ -1485,8 +1524,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int qi = 0; qi < (halves_done ? 0 : NQW); ++qi) {
           const int n = st->cnt[par][qi];
           const int64_t t = tq0 + qi;
-          if (kDefer && fin && etid == 0 && t >= p.S) bars->jobs[set][eg][qi] = make_uint4(0u, 0u, 0u, kJobSkip);
-          if (fin ? t >= p.S : n <= cut_min) continue;
+          if (kDefer && fin && etid == 0 && t >= t_end) bars->jobs[set][eg][qi] = make_uint4(0u, 0u, 0u, kJobSkip);
+          if (fin ? t >= t_end : n <= cut_min) continue;
           if (!fin) {
             uint2* buf = cand + qi * static_cast<size_t>(p.cap);
             int kept;
@@ -1543,7 +1582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               const float sc = key_to_float(k);
               if (m == 1) {
-                __stcs(&orow[pos], static_cast<int32_t>(ix));
+                __stcs(&orow[pos], static_cast<int32_t>(ix) + out_shift);
                 if (srow) srow[pos] = sc;
               } else {
                 for (int rr = 0; rr < m; ++rr) {
@@ -1602,7 +1641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int len = kept * m;
             if (m > 1) {
-              const int64_t g = p.q_pos0 + t;
+              const int64_t g = t + pos_shift;
               const int tail = static_cast<int>((g + 1) % m);
               const int64_t first = g + 1 - tail;
               for (int i = etid; i < tail; i += kBM) {
@@ -1653,6 +1692,12 @@ void fill_variant(ScoreVariant* v) {
   using C = Cfg<H, D, FP8>;
   v->fn = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8, PRUNE, false>);
   v->fn_split = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8, PRUNE, true>);
+  // the segmented instance serves packed documents without the pruning
+  // certificate (whose key norms are numbered over a single problem's keys)
+  if constexpr (!PRUNE)
+    v->fn_seg = reinterpret_cast<const void*>(&score_topk_kernel<H, D, FP8, false, false, true>);
+  else
+    v->fn_seg = nullptr;
   v->queries_per_block = C::QB;
   v->queries_per_wg = C::NQW;
   v->groups = kEpiGroups;

@@ -274,9 +274,12 @@ indexer_status indexer_topk_witness(const indexer_problem* p, const void* q, con
  * and doc_bounds[n_docs] within the keys.  Other arguments, output layout
  * (global positions, -1 padding, lengths) and errors as indexer_topk; the
  * workspace is indexer_docs_workspace_bytes bytes, and indexer_read_status
- * covers all documents.  Each document runs as its own indexer call on
- * `stream` (a few short documents are therefore cheaper batched into one
- * problem without bounds). */
+ * covers all documents.  A batch of many short token or compressed-key
+ * documents (more query blocks than half the SMs, fewer than two per SM per
+ * document on average; no INDEXER_FLAG_PRUNE) runs as ONE launch over a table
+ * of every document's query blocks, copied into the workspace from host
+ * memory; otherwise (pooled keys, pruning, long documents, a few queries)
+ * each document runs as its own indexer call on `stream`. */
 indexer_status indexer_docs_workspace_bytes(const indexer_problem* p, const int64_t* doc_bounds,
                                             int32_t n_docs, size_t* bytes);
 indexer_status indexer_topk_docs(const indexer_problem* p, const void* q, const void* k,

@@ -75,6 +75,50 @@ def test_docs_gaussian(cuda_ok, wl, bounds):
         assert ((row >= bounds[d]) & (row <= g)).all()
 
 
+def _random_bounds(total, lo, hi, seed):
+    """Document bounds of random lengths in [lo, hi] covering [0, total)."""
+    rng = np.random.default_rng(seed)
+    b = [0]
+    while b[-1] < total:
+        b.append(min(total, b[-1] + int(rng.integers(lo, hi + 1))))
+    return b
+
+
+# Batches with many query blocks run as one launch over a table of every
+# document's blocks (the per-launch cost dominates short documents); these
+# cover it for one-query (H = 64, 4), two-query (H = 32) and FP8 groups.
+@pytest.mark.parametrize("wl,lengths", [
+    (W.Workload("docs_many_h4", S=900, T=900, H=4, D=64, K=8, seed=89, values="int"), (1, 12)),
+    (W.Workload("docs_many_h32", S=1200, T=1200, H=32, D=128, K=32, seed=87, values="int"), (1, 40)),
+    (W.Workload("docs_many_csa", S=2000, T=500, H=64, D=128, K=16, visibility=W.COMPRESSED, ratio=4, seed=90,
+                values="int"), (4, 60)),
+], ids=lambda x: x.name if isinstance(x, W.Workload) else "")
+def test_docs_one_launch_integer_bit_exact(cuda_ok, wl, lengths):
+    key_tokens = wl.T * wl.ratio if wl.visibility == W.COMPRESSED else wl.T
+    bounds = _random_bounds(key_tokens, *lengths, seed=wl.seed)
+    if wl.visibility == W.COMPRESSED:   # documents start on whole compressed keys
+        bounds = sorted(set([0] + [x // wl.ratio * wl.ratio for x in bounds[1:-1]] + [key_tokens]))
+    inp = W.generate(wl, "cuda")
+    gpu = _run_docs(wl, inp, bounds)
+    ref = _oracle_docs(wl, inp, bounds)
+    parity.assert_exact(gpu, ref, np.arange(wl.S))
+
+
+def test_docs_one_launch_fp8(cuda_ok):
+    wl = W.Workload("docs_fp8", S=800, T=800, H=64, D=128, K=64, dtype="fp8", seed=88)
+    bounds = _random_bounds(wl.T, 10, 120, seed=88)
+    inp = W.generate(wl, "cuda")
+    gpu = _run_docs(wl, inp, bounds)
+    ref = _oracle_docs(wl, inp, bounds)
+    recall = parity.assert_tolerant(wl, gpu, ref, np.arange(wl.S))
+    assert recall >= 0.9999
+    gi, gl = gpu[0].cpu().numpy(), gpu[1].cpu().numpy()
+    for r in range(wl.S):
+        d = int(np.searchsorted(bounds, r, side="right")) - 1
+        row = gi[r, : gl[r]]
+        assert ((row >= bounds[d]) & (row <= r)).all()
+
+
 def test_docs_reject_bad_bounds(cuda_ok):
     from head_weighted_relu_b200 import indexer as I
     prob = I.make_problem(100, 100, 64, 128, 16)
