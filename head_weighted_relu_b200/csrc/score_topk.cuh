@@ -15,7 +15,8 @@
 // accumulator: 4 for 64 heads, 8 for 32, ...) at a time:
 //   warp 0      TMA producer: the block's q rows once, then key tiles of 128
 //               rows through a ring of shared-memory stages;
-//   warp 1      MMA issuer: key tile n goes to accumulator n & 1,
+//   warp 1      MMA issuer: key tile n goes to accumulator n % NACC (two
+//               at N = 256, four at N = 128: as many as TMEM's columns hold),
 //               acc[key, (query, head)] = k_tile . q_block^T
 //               (M = 128 keys = TMEM lanes, N = queries x heads <= 256 columns,
 //               K = D), tcgen05.mma with FP32 accumulation in TMEM, so the
@@ -1091,7 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t kph = 0, qf_ph = 0;
       uint32_t ae_ph[4] = {0u, 0u, 0u, 0u};
-      uint32_t tcount = 0;  // tiles issued so far; tile n goes to accumulator n & 1
+      uint32_t tcount = 0;  // tiles issued so far; tile n goes to accumulator n % NACC
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const Item it = item_of<QB, SPLIT, SEG>(p, r, blockIdx.x, gridDim.x);
@@ -1155,7 +1156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------- output-row writers
     // Warps 2 and 3 write the output rows of each finished query block while
     // the epilogue groups go on with the next block: a group hands over its
-    // queries' candidate buffers (one of two sets) with their final cuts.
+    // queries' candidate buffers (one of kSets sets) with their final cuts.
     const int ww = warp - 2;
     for (int r = 0;; ++r) {
       const Item it = item_of<QB, SPLIT, SEG>(p, r, blockIdx.x, gridDim.x);
@@ -1231,7 +1232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool kDefer = !SPLIT && !FP8;
     volatile int* cut_round = &bars->cut_round;
     volatile int* seen = &bars->seen[eg];
-    uint32_t tcount = 0;    // tiles drained so far; tile n sits in accumulator n & 1
+    uint32_t tcount = 0;    // tiles drained so far; tile n sits in accumulator n % NACC
     int par = 0;
     bool failed = false;
     unsigned long long n_screened = 0ull, n_bounded = 0ull, n_skipped = 0ull;  // pruning counters (lane 0)
