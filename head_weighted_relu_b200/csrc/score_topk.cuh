@@ -21,6 +21,10 @@
 //               (M = 128 keys = TMEM lanes, N = queries x heads <= 256 columns,
 //               K = D), tcgen05.mma with FP32 accumulation in TMEM, so the
 //               next tile's product overlaps the epilogue of this one;
+//   warps 2, 3  row writers (bf16 single-range instances): they write the
+//               output rows of a finished block from its candidate buffers
+//               and final cuts while the epilogue goes on with the next
+//               block (buffers rotate through kSets sets);
 //   warps 4..19 four epilogue warpgroups, each owning a quarter of the
 //               columns (whole queries).  A warpgroup keeps its queries' head
 //               weights in registers for the whole block, so the head sum
@@ -32,9 +36,16 @@
 //               running threshold to a per-query candidate buffer in global
 //               memory -- in key order, so the buffer is always sorted by key
 //               index.  A buffer about to overflow is cut back toward its
-//               top-K by a warpgroup radix select, which raises the threshold.
+//               top-K by a warpgroup radix select, which raises the threshold
+//               (bf16: groups whose buffers fill cut together, in rounds).
 //               After the block's last tile the same select gives the final
-//               top-K, written in key order.
+//               top-K, written in key order by the row writers (or by the
+//               group itself: FP8 and split key ranges).
+//
+// Instances: SPLIT cuts each block's key tiles into ranges merged afterwards
+// (decode-like shapes); SEG takes its query blocks from a table spanning the
+// documents of a packed batch (each block's rows, visibility origin and
+// keys), so that many short documents run as one launch.
 //
 // Keys arrive in ascending index order, so once a buffer holds the top-K of
 // the keys seen so far with K-th entry (v, i), a later key (index > i) can
@@ -50,7 +61,7 @@
 
 namespace hwr {
 
-// 20 warps: warpgroup 0 = TMA producer, MMA issuer and two idle warps;
+// 20 warps: warpgroup 0 = TMA producer, MMA issuer and two row writers;
 // warpgroups 1..4 = epilogue.  Registers at launch: 640 x 96 = 61,440.
 // Warpgroup 0 drops to 32 per thread and the epilogue takes 112:
 // 128 x 32 + 512 x 112 = 61,440 (per SMSP: 32*32 + 4*112*32 = 15,360 <= 16,384).
